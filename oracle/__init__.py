@@ -1,0 +1,196 @@
+"""CPU oracle for quantized video-DiT self-attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product library never routes through it and
+shares no code with it.
+
+What it computes is stated in ``oracle.c`` (a plain, slow C restatement of the
+method of page 1 of the TMAP / Taobao Faxiang image-to-video write-up,
+"Attention performance optimisation": SageAttention-style INT8 QK^T with K
+smoothing and a zero-scale guard, FP8 P.V, online softmax, and a per-layer
+BF16 table).  This module compiles it in-tree and wraps it with numpy.
+
+Every function here is pinned by ``tests/test_oracle_*.py`` against things
+other than itself: exact rational brute force, the OCP FP8 code table,
+closed-form special cases and invariants of exact softmax attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+TILE = 128
+# emulation switches (see orc_attn_emul): used only to pin the emulation
+EMUL_P_FP32 = 1
+EMUL_V_EXACT = 2
+EMUL_QK_EXACT = 4
+EMUL_ONE_TILE = 8
+
+
+def build(force: bool = False) -> str:
+    """Compiles oracle.c into liboracle.so (gcc -O2, OpenMP, no contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _p(a, ct):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i32, i64 = ctypes.c_int, ctypes.c_long
+            P = ctypes.POINTER
+            u16, i8, u8, f32, f64, s32 = (P(ctypes.c_uint16), P(ctypes.c_int8), P(ctypes.c_uint8),
+                                          P(ctypes.c_float), P(ctypes.c_double), P(ctypes.c_int32))
+            lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_decode.restype = ctypes.c_double
+            lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.orc_e4m3_encode.restype = ctypes.c_uint8
+            lib.orc_k_mean.argtypes = [u16, i32, i32, i32, i32, f32]
+            lib.orc_quant_int8_blocks.argtypes = [u16, f32, i32, i32, i32, i32, i8, f32]
+            lib.orc_quant_v_fp8.argtypes = [u16, i32, i32, i32, i32, u8, f32]
+            lib.orc_qk_tile.argtypes = [i8, i8, i32, i32, i64, i32, i32, s32]
+            lib.orc_attn_exact.argtypes = [u16, u16, u16, i32, i32, i32, i32, P(i32), i32, f64]
+            lib.orc_attn_emul.argtypes = [i8, f32, i8, f32, u8, f32, i32, i32, i32, i32, P(i32), i32, i32,
+                                          u16, u16, u16, f32, u16]
+            lib.orc_layer_schedule.argtypes = [i32, P(i32), i32, i8]
+            lib.orc_layer_schedule.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+# ---------------- FP8 e4m3 ----------------
+
+def e4m3_decode(code: int) -> float:
+    return _load().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(x: float) -> int:
+    return int(_load().orc_e4m3_encode(float(x)))
+
+
+def e4m3_decode_table() -> np.ndarray:
+    """fp64 value of each of the 256 e4m3 codes (NaN for 0x7F / 0xFF)."""
+    return np.array([e4m3_decode(i) for i in range(256)], dtype=np.float64)
+
+
+# ---------------- prepass (a1..a4) ----------------
+
+def k_mean(k: np.ndarray) -> np.ndarray:
+    """a1: fp32 [B,H,d] per-channel token mean of bf16 K [B,H,N,d]."""
+    k = _c(k, np.uint16)
+    B, H, N, d = k.shape
+    out = np.empty((B, H, d), dtype=np.float32)
+    _load().orc_k_mean(_p(k, ctypes.c_uint16), B, H, N, d, _p(out, ctypes.c_float))
+    return out
+
+
+def quant_int8_blocks(x: np.ndarray, mean: np.ndarray | None = None):
+    """a2/a3: per-128-token-block INT8 codes [B,H,N,d] and fp32 scales [B,H,nblk]."""
+    x = _c(x, np.uint16)
+    B, H, N, d = x.shape
+    nb = (N + TILE - 1) // TILE
+    codes = np.empty((B, H, N, d), dtype=np.int8)
+    scale = np.empty((B, H, nb), dtype=np.float32)
+    m = None if mean is None else _c(mean, np.float32)
+    _load().orc_quant_int8_blocks(_p(x, ctypes.c_uint16), _p(m, ctypes.c_float), B, H, N, d,
+                                  _p(codes, ctypes.c_int8), _p(scale, ctypes.c_float))
+    return codes, scale
+
+
+def quant_v_fp8(v: np.ndarray):
+    """a4: e4m3 codes [B,H,N,d] (natural layout) and fp32 per-channel scales [B,H,d]."""
+    v = _c(v, np.uint16)
+    B, H, N, d = v.shape
+    codes = np.empty((B, H, N, d), dtype=np.uint8)
+    scale = np.empty((B, H, d), dtype=np.float32)
+    _load().orc_quant_v_fp8(_p(v, ctypes.c_uint16), B, H, N, d, _p(codes, ctypes.c_uint8),
+                            _p(scale, ctypes.c_float))
+    return codes, scale
+
+
+def prepass(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
+    """a1..a4 in order; returns every intermediate the path exposes."""
+    mean = k_mean(k)
+    q8, qs = quant_int8_blocks(q)
+    k8, ks = quant_int8_blocks(k, mean)
+    v8, vs = quant_v_fp8(v)
+    return dict(k_mean=mean, q_i8=q8, q_scale=qs, k_i8=k8, k_scale=ks, v_f8=v8, v_scale=vs)
+
+
+def qk_tile(q8: np.ndarray, k8: np.ndarray, bh: int, qb: int, kb: int) -> np.ndarray:
+    """a5: exact int32 [128,128] tile of Q_i8 K_i8^T for one (b*H+h, q-block, k-block)."""
+    q8 = _c(q8, np.int8)
+    k8 = _c(k8, np.int8)
+    B, H, N, d = q8.shape
+    out = np.empty((TILE, TILE), dtype=np.int32)
+    _load().orc_qk_tile(_p(q8, ctypes.c_int8), _p(k8, ctypes.c_int8), N, d, bh, qb, kb,
+                        _p(out, ctypes.c_int32))
+    return out
+
+
+# ---------------- attention ----------------
+
+def attn_exact(q, k, v, rows=None) -> np.ndarray:
+    """O1: fp64 softmax(Q K^T/sqrt(d)) V for the given query rows, shape [B,H,len(rows),d]."""
+    q, k, v = (_c(a, np.uint16) for a in (q, k, v))
+    B, H, N, d = q.shape
+    rows = np.arange(N, dtype=np.int32) if rows is None else _c(np.asarray(rows, dtype=np.int32), np.int32)
+    out = np.empty((B, H, len(rows), d), dtype=np.float64)
+    _load().orc_attn_exact(_p(q, ctypes.c_uint16), _p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
+                           B, H, N, d, _p(rows, ctypes.c_int), len(rows), _p(out, ctypes.c_double))
+    return out
+
+
+def attn_emul(pre: dict, rows=None, flags: int = 0, q=None, k=None, v=None):
+    """O2: emulated quantized attention for the given rows.
+
+    Returns (fp32 values [B,H,R,d] before output rounding, bf16 bits [B,H,R,d]).
+    """
+    q8, k8, v8 = _c(pre["q_i8"], np.int8), _c(pre["k_i8"], np.int8), _c(pre["v_f8"], np.uint8)
+    qs, ks, vs = (_c(pre[n], np.float32) for n in ("q_scale", "k_scale", "v_scale"))
+    B, H, N, d = q8.shape
+    rows = np.arange(N, dtype=np.int32) if rows is None else _c(np.asarray(rows, dtype=np.int32), np.int32)
+    out = np.empty((B, H, len(rows), d), dtype=np.float32)
+    outb = np.empty((B, H, len(rows), d), dtype=np.uint16)
+    qb_, kb_, vb_ = (None if a is None else _c(a, np.uint16) for a in (q, k, v))
+    _load().orc_attn_emul(_p(q8, ctypes.c_int8), _p(qs, ctypes.c_float), _p(k8, ctypes.c_int8),
+                          _p(ks, ctypes.c_float), _p(v8, ctypes.c_uint8), _p(vs, ctypes.c_float),
+                          B, H, N, d, _p(rows, ctypes.c_int), len(rows), int(flags),
+                          _p(qb_, ctypes.c_uint16), _p(kb_, ctypes.c_uint16), _p(vb_, ctypes.c_uint16),
+                          _p(out, ctypes.c_float), _p(outb, ctypes.c_uint16))
+    return out, outb
+
+
+def layer_schedule(num_layers: int, fp_layers) -> np.ndarray:
+    """a11: int8 modes [num_layers]: 0 = BF16 for the listed layers, 1 = INT8/FP8 otherwise."""
+    fp = np.asarray(list(fp_layers), dtype=np.int32)
+    modes = np.empty(max(num_layers, 0), dtype=np.int8)
+    rc = _load().orc_layer_schedule(num_layers, _p(fp, ctypes.c_int), len(fp), _p(modes, ctypes.c_int8))
+    if rc != 0:
+        raise ValueError("layer index out of range")
+    return modes
