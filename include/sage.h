@@ -1,0 +1,188 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) quantized self-attention library for
+ * video diffusion transformers.
+ *
+ * The operation is the full-sequence self-attention of a video DiT, which
+ * page 1 of the TMAP / Taobao Faxiang image-to-video write-up
+ * (ai.aiking123.com/155823.html, section "Attention performance
+ * optimisation / Background") profiles as aten.scaled_dot_product_flash_attention
+ * (73.76% of the model's FLOPs, 72% of runtime), and which it replaces by the
+ * SageAttention operator ("attention quantization"), keeping some layers at
+ * original precision ("keeping video quality") and guarding the per-channel
+ * quantization coefficient against all-zero channels ("operator details").
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are row-major [B, H, N, d] ("BHND"): tokens contiguous per head,
+ *    channels contiguous per token.  d must be 64 or 128, N >= 1, B, H >= 1,
+ *    B * H * ceil(N/128) * 128 * d < 2^31.
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  Device
+ *    pointers must be 16-byte aligned.  The caller owns all memory; the
+ *    library allocates nothing and keeps no state between calls.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls are asynchronous on that stream; no call synchronises except
+ *    sage_status().
+ *  - Every function returns SAGE_OK (0) or a negative SAGE_E* code; none
+ *    aborts or throws.  Argument errors are detected on the host before any
+ *    launch.  Device-side failures (a bounded wait that ran out) are recorded
+ *    in the status word inside the workspace and reported by sage_status().
+ */
+#ifndef SAGE_H
+#define SAGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* attention modes (one per layer, see attn_layer_schedule) */
+#define SAGE_MODE_BF16 0      /* exact softmax attention, BF16 tensor-core MMAs */
+#define SAGE_MODE_INT8_FP8 1  /* smoothed INT8 QK^T, FP8 e4m3 P.V             */
+
+/* status codes */
+#define SAGE_OK 0
+#define SAGE_EINVAL (-1)        /* bad size, null or misaligned pointer, bad mode      */
+#define SAGE_EUNSUPPORTED (-2)  /* d not in {64,128}, or the device is not sm_100     */
+#define SAGE_ELAUNCH (-3)       /* a CUDA launch or runtime call failed               */
+#define SAGE_EWORKSPACE (-4)    /* workspace smaller than sage_workspace_bytes()      */
+#define SAGE_ETIMEOUT (-5)      /* a bounded device-side wait ran out (see sage_status) */
+
+/* tile sizes of the quantization blocks and of the attention tiles */
+#define SAGE_BLK_Q 128
+#define SAGE_BLK_K 128
+/* static scale of the FP8 P operand: P8 = e4m3(p * 448), p in [0, 1] */
+#define SAGE_P_SCALE 448.0f
+
+/*
+ * Bytes of device workspace sage_attn_fwd needs for (B, H, N, d, mode).
+ * INT8_FP8: the quantized Q/K/V, their scales, the K mean, prepass partials
+ * and a 256-byte status word.  BF16: the status word only.
+ * Returns 0 for invalid arguments.
+ */
+size_t sage_workspace_bytes(int B, int H, int N, int d, int mode);
+
+/*
+ * Quantization prepass (steps a1-a4 of the scheme), fused into three kernels:
+ *  a1  k_mean[b,h,c] = (1/N) sum_n K[b,h,n,c] (fp64 sums in a fixed order,
+ *      rounded once to fp32);
+ *  a2  Ks = fp32(K) - k_mean; per 128-token block: amax = max|Ks|,
+ *      k_scale = amax/127, k_i8 = clamp(rne(Ks * (127/amax)), -127, 127);
+ *  a3  the same for Q without smoothing;
+ *  a4  per channel amax over all tokens of V, v_scale = amax/448,
+ *      v_f8t = e4m3_rne_satfinite(V * (448/amax)), stored transposed.
+ * An all-zero block or channel (amax == 0) gets scale 0 and all-zero codes:
+ * no division by zero, no NaN (the fix described under "operator details").
+ *
+ * q, k, v   bf16 [B,H,N,d]                                  (input)
+ * q_i8      int8 [B,H,nQ*128,d], rows >= N zero              (output)
+ * q_scale   fp32 [B,H,nQ]                                    (output)
+ * k_i8      int8 [B,H,nK*128,d], rows >= N zero              (output)
+ * k_scale   fp32 [B,H,nK]                                    (output)
+ * k_mean    fp32 [B,H,d]                                     (output)
+ * v_f8t     e4m3 [B,H,d,nK*128], token-contiguous, cols >= N zero (output)
+ * v_scale   fp32 [B,H,d]                                     (output)
+ * scratch   device scratch of sage_prepass_scratch_bytes() bytes (partials)
+ * with nQ = nK = ceil(N/128).
+ */
+size_t sage_prepass_scratch_bytes(int B, int H, int N, int d);
+int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                     int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                     uint8_t* v_f8t, float* v_scale, void* scratch, size_t scratch_bytes,
+                     void* stream);
+
+/*
+ * Attention over already-quantized operands (steps a5-a9): per 128x128 tile
+ * S = Q_i8 K_i8^T in exact int32 (tcgen05 kind::i8), s = S * q_scale * k_scale
+ * * log2(e)/sqrt(d), keys >= N masked, online softmax with p = 2^(s - m),
+ * P8 = e4m3(p * 448) kept in tensor memory, O += P8 V8 (tcgen05 kind::f8f6f4,
+ * fp32), O = O * v_scale / (448 * l) rounded to bf16.
+ * Operands as written by sage_quantize_qk; o is bf16 [B,H,N,d] (output).
+ * status: a 256-byte device status region (e.g. the start of a workspace);
+ * failures are OR-ed into its first word.
+ */
+int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                        const float* k_scale, const uint8_t* v_f8t, const float* v_scale,
+                        void* o, int B, int H, int N, int d, void* status, void* stream);
+
+/*
+ * Full-sequence self-attention O = softmax(Q K^T / sqrt(d)) V, non-causal,
+ * q, k, v, o bf16 [B,H,N,d].
+ * mode SAGE_MODE_INT8_FP8: sage_quantize_qk into the workspace, then
+ *   sage_attn_quantized.
+ * mode SAGE_MODE_BF16: S = Q K^T with BF16 tensor-core MMAs (fp32
+ *   accumulate), online softmax in fp32, P rounded to bf16, O += P V
+ *   (fp32), O / l rounded to bf16.  Uses only the status word of the workspace.
+ * workspace: device buffer of at least sage_workspace_bytes(B,H,N,d,mode)
+ * bytes, 256-byte aligned; its first 256 bytes are the status word.
+ */
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                  int mode, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Per-layer mode table for selective quantization ("keeping video quality":
+ * some attention layers stay at original precision at every denoising step).
+ * full_precision_layers (host, n_fp entries, duplicates allowed) -> BF16,
+ * every other layer -> INT8_FP8.  modes_out: host int8 [num_layers].
+ * Returns SAGE_EINVAL if an index is outside [0, num_layers).
+ */
+int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_fp, int8_t* modes_out);
+
+/*
+ * Reads and clears the device status word at the start of `workspace`
+ * (synchronises `stream`).  Returns SAGE_OK, SAGE_ETIMEOUT if a bounded
+ * device-side wait ran out since the last call, or SAGE_ELAUNCH if the stream
+ * reports a CUDA error.
+ */
+int sage_status(void* workspace, void* stream);
+
+/* Human-readable text of a status code (static storage). */
+const char* sage_strerror(int code);
+
+/*
+ * Returns SAGE_OK if the current device is an sm_100 part the kernels were
+ * built for, SAGE_EUNSUPPORTED otherwise, SAGE_ELAUNCH if no device is usable.
+ */
+int sage_device_check(void);
+
+/*
+ * Diagnostic: copies int32 QK^T tiles computed by the same TMA + tcgen05
+ * kind::i8 path the attention kernel uses.  q_i8, k_i8 as written by
+ * sage_quantize_qk; tile_list: device int32 [n][4] of (b, h, qb, kb);
+ * out: device int32 [n, 128, 128], out[t][i][j] = S[qb*128+i, kb*128+j].
+ */
+int sage_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int B, int H, int N, int d,
+                      const int* tile_list, int n, int32_t* out, void* stream);
+
+/*
+ * Diagnostic: one 128-row P.V product through the same operand path as the
+ * attention kernels, with P written to tensor memory from registers.
+ * mode INT8_FP8: p (device, e4m3 [128,128]) times vt (device, e4m3 [d,128],
+ *   key-contiguous) -> out fp32 [128,d] = sum_j p[i,j] * vt[c,j].
+ * mode BF16: p (device, bf16 [128,128]) times vt (device, bf16 [128,d],
+ *   channel-contiguous, i.e. V itself) -> out fp32 [128,d].
+ */
+int sage_dbg_pv_tile(const void* p, const void* vt, int d, int mode, float* out, void* stream);
+
+/*
+ * Diagnostic: one 128x128 BF16 QK^T tile through the BF16 attention path's
+ * operand staging.  q, k: device bf16 [128,d]; out fp32 [128,128].
+ */
+int sage_dbg_qk_bf16_tile(const void* q, const void* k, int d, float* out, void* stream);
+
+/*
+ * Test hook of the bounded-wait machinery: runs the quantized attention
+ * kernel on the given operands with a wait that no one satisfies and a wait
+ * limit of `timeout_cycles` SM clocks, so that the kernel records
+ * SAGE_ETIMEOUT in `status` and returns without hanging.  Same operands as
+ * sage_attn_quantized.
+ */
+int sage_dbg_attn_forced_timeout(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                 const float* k_scale, const uint8_t* v_f8t, const float* v_scale,
+                                 void* o, int B, int H, int N, int d, void* status,
+                                 long long timeout_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_H */

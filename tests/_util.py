@@ -1,0 +1,61 @@
+"""Shared helpers of the parity tests: metrics and head-sliced oracle calls."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+
+# Tolerances of the path (quantized vs emulation, quantized vs exact, bf16 vs exact)
+COS_EMUL = 0.9999
+MAXABS_EMUL = 5e-3          # x max|V| of the head
+COS_EXACT = 0.995
+REL_L2_BF16 = 4e-3
+
+
+def cos(a, b) -> float:
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
+    na, nb = np.linalg.norm(a), np.linalg.norm(b)
+    if na == 0 and nb == 0:
+        return 1.0
+    return float(a @ b / (na * nb))
+
+
+def rel_l2(got, want) -> float:
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    return float(np.linalg.norm(got - want) / np.linalg.norm(want))
+
+
+def bf16_to_np(t) -> np.ndarray:
+    """torch bf16 tensor -> fp32 numpy."""
+    import torch
+    return t.detach().to("cpu").view(torch.int16).numpy().view(np.uint16).astype(np.uint32).__lshift__(16).view(np.float32)
+
+
+def heads(a: np.ndarray, hs) -> np.ndarray:
+    """Contiguous [B, len(hs), N, d] slice of a [B, H, N, d] array."""
+    return np.ascontiguousarray(a[:, list(hs)])
+
+
+def small_workloads():
+    """Ragged and degenerate shapes the oracle finishes in seconds."""
+    W = synth.Workload
+    return [
+        synth.WORKLOADS["tiny"],
+        W("n1", 1, 1, 1, 128, seed=21),
+        W("n127_d64", 1, 2, 127, 64, seed=22),
+        W("n129", 1, 3, 129, 128, seed=23, zero_k_channel=7),
+        W("n1000_d64_b2", 2, 2, 1000, 64, seed=24, outlier_frac=0.01),
+        W("n640_outlier", 1, 2, 640, 128, seed=25, outlier_frac=0.01),
+        W("n385", 1, 1, 385, 128, seed=26, k_off_std=0.0),
+    ]
+
+
+def emul_and_exact(q, k, v, rows):
+    """Oracle prepass + O2 (fp32) and O1 (fp64) for the given rows of every head."""
+    pre = oracle.prepass(q, k, v)
+    o2, _ = oracle.attn_emul(pre, rows)
+    o1 = oracle.attn_exact(q, k, v, rows)
+    return pre, o2, o1

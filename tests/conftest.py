@@ -18,3 +18,30 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def big_inputs(cuda_dev):
+    """Full-size seeded inputs of a named workload: host bf16 bits + device copies.
+
+    Keeps only the most recently requested workload alive to bound memory.
+    """
+    import numpy as np
+    import torch
+
+    import synth
+
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            w = synth.WORKLOADS[name]
+            q, k, v = synth.qkv_numpy(w)
+            dev = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(cuda_dev) for a in (q, k, v)]
+            cache[name] = (q, k, v, *dev)
+        return cache[name]
+
+    yield get
+    cache.clear()

@@ -1,0 +1,67 @@
+"""The C-ABI library loads, exports every symbol include/sage.h declares, and
+rejects bad arguments on the host before touching a device (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from video_dit_quantized_b200 import sage
+
+EXPECTED = {
+    "sage_workspace_bytes", "sage_prepass_scratch_bytes", "sage_quantize_qk", "sage_attn_quantized",
+    "sage_attn_fwd", "attn_layer_schedule", "sage_status", "sage_strerror", "sage_device_check",
+    "sage_dbg_qk_tiles", "sage_dbg_pv_tile", "sage_dbg_qk_bf16_tile", "sage_dbg_attn_forced_timeout",
+}
+
+
+def test_header_declares_the_expected_entry_points():
+    assert set(sage.header_functions()) == EXPECTED
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(sage._build.LIB_PATH)
+    for name in sage.header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_workspace_sizes():
+    # BF16 mode needs only the status word
+    assert sage.workspace_bytes(1, 2, 1024, 128, sage.MODE_BF16) == 256
+    # INT8/FP8: Q_i8 + K_i8 + V_f8t dominate (3 bytes per element of the padded tensor)
+    B, H, N, d = 1, 40, 75600, 128
+    npad = (N + 127) // 128 * 128
+    ws = sage.workspace_bytes(B, H, N, d, sage.MODE_INT8_FP8)
+    assert 3 * B * H * npad * d < ws < 3 * B * H * npad * d * 1.1
+    for bad in [(0, 1, 8, 128), (1, 0, 8, 128), (1, 1, 0, 128), (1, 1, 8, 96), (1, 70000, 8, 64)]:
+        assert sage.workspace_bytes(*bad, sage.MODE_INT8_FP8) == 0
+    assert sage.workspace_bytes(1, 1, 8, 128, 7) == 0
+
+
+def test_argument_errors_are_host_side():
+    vp = ctypes.c_void_p
+    lib = sage.LIB
+    fake = vp(0x100000)         # never dereferenced: validation fails first
+    # bad head dim -> unsupported, before any device work
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 1, 128, 96, 0, fake, 1 << 20, None) == sage.EUNSUPPORTED
+    # N = 0, null pointer, misaligned pointer, bad mode
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 1, 0, 128, 0, fake, 1 << 20, None) == sage.EINVAL
+    assert lib.sage_attn_fwd(None, fake, fake, fake, 1, 1, 128, 128, 0, fake, 1 << 20, None) == sage.EINVAL
+    assert lib.sage_attn_fwd(vp(0x100008), fake, fake, fake, 1, 1, 128, 128, 0, fake, 1 << 20, None) == sage.EINVAL
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 1, 128, 128, 5, fake, 1 << 20, None) == sage.EINVAL
+    # workspace too small
+    assert lib.sage_attn_fwd(fake, fake, fake, fake, 1, 1, 128, 128, 1, fake, 1000, None) == sage.EWORKSPACE
+    # prepass with too little scratch
+    assert lib.sage_quantize_qk(*([fake] * 3), 1, 1, 128, 128, *([fake] * 8), 16, None) == sage.EWORKSPACE
+
+
+def test_layer_schedule_host():
+    assert sage.layer_schedule(40, (0, 8, 16, 24, 32)) == [0 if l % 8 == 0 else 1 for l in range(40)]
+    assert sage.layer_schedule(3, [2, 2]) == [1, 1, 0]
+    with pytest.raises(sage.SageError):
+        sage.layer_schedule(4, [4])
+    with pytest.raises(sage.SageError):
+        sage.layer_schedule(4, [-1])
+
+
+def test_strerror_covers_codes():
+    for c in (0, -1, -2, -3, -4, -5):
+        assert sage.strerror(c) and sage.strerror(c) != "unknown status"

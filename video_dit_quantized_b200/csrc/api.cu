@@ -1,0 +1,274 @@
+// api.cu -- the extern "C" entry points declared in include/sage.h: argument
+// validation, workspace layout, TMA tensor-map encoding and kernel launches.
+// Marshalling only; every step of the computation runs in the kernels of
+// prepass.cu and attention.cu.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sage.h"
+#include "internal.h"
+
+namespace sage {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace layout of the INT8/FP8 mode; every region 256-byte aligned.
+struct Layout {
+  size_t status, q_i8, k_i8, v_f8t, q_scale, k_scale, k_mean, v_scale, scratch, total;
+};
+
+Layout layout(int B, int H, int N, int d) {
+  const size_t BH = (size_t)B * H, nT = num_tiles(N), Npad = nT * kTile;
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes, 256);
+    return at;
+  };
+  L.status = take(256);
+  L.q_i8 = take(BH * Npad * d);
+  L.k_i8 = take(BH * Npad * d);
+  L.v_f8t = take(BH * d * Npad);
+  L.q_scale = take(BH * nT * 4);
+  L.k_scale = take(BH * nT * 4);
+  L.k_mean = take(BH * d * 4);
+  L.v_scale = take(BH * d * 4);
+  L.scratch = take(prepass_scratch_bytes((int)BH, N, d));
+  L.total = off;
+  return L;
+}
+
+int check_shape(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return SAGE_EINVAL;
+  if (d != 64 && d != 128) return SAGE_EUNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 65535) return SAGE_EINVAL;                       // grid.y limit
+  const long long Npad = (long long)num_tiles(N) * kTile;
+  if (BH * Npad * d >= (1LL << 31)) return SAGE_EINVAL;     // 32-bit TMA coordinates / offsets
+  return SAGE_OK;
+}
+
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ELAUNCH;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SAGE_ELAUNCH;
+  return (major == 10 && minor == 0) ? SAGE_OK : SAGE_EUNSUPPORTED;
+}
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE_OK;
+  if (e == cudaErrorInvalidValue) return SAGE_EINVAL;
+  return SAGE_ELAUNCH;
+}
+
+}  // namespace
+
+bool encode_tmap_2d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {outer_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(static_cast<CUtensorMap*>(map), dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_tmap_3d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
+                    CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box0, box1, box2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(static_cast<CUtensorMap*>(map), dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace sage
+
+using namespace sage;
+
+extern "C" {
+
+size_t sage_workspace_bytes(int B, int H, int N, int d, int mode) {
+  if (check_shape(B, H, N, d) != SAGE_OK) return 0;
+  if (mode == SAGE_MODE_BF16) return 256;
+  if (mode == SAGE_MODE_INT8_FP8) return layout(B, H, N, d).total;
+  return 0;
+}
+
+size_t sage_prepass_scratch_bytes(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d) != SAGE_OK) return 0;
+  return prepass_scratch_bytes(B * H, N, d);
+}
+
+int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, int N, int d, int8_t* q_i8,
+                     float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t, float* v_scale,
+                     void* scratch, size_t scratch_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  const void* ptrs[] = {q, k, v, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if (scratch_bytes < prepass_scratch_bytes(B * H, N, d)) return SAGE_EWORKSPACE;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  const PrepassScratch s = prepass_scratch_carve(scratch, B * H, N, d);
+  return launch_status(launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale,
+                                      s, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                        const uint8_t* v_f8t, const float* v_scale, void* o, int B, int H, int N, int d, void* status,
+                        void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  const void* ptrs[] = {q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, status};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d,
+                                        static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int mode,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8) return SAGE_EINVAL;
+  const void* ptrs[] = {q, k, v, o, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_EINVAL;
+  if (workspace_bytes < sage_workspace_bytes(B, H, N, d, mode)) return SAGE_EWORKSPACE;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  if (mode == SAGE_MODE_BF16)
+    return launch_status(launch_attn_bf16(q, k, v, o, B * H, N, d, status, kDefaultTimeoutCycles, st));
+  const Layout L = layout(B, H, N, d);
+  auto q_i8 = reinterpret_cast<int8_t*>(ws + L.q_i8);
+  auto k_i8 = reinterpret_cast<int8_t*>(ws + L.k_i8);
+  auto v_f8t = reinterpret_cast<uint8_t*>(ws + L.v_f8t);
+  auto q_scale = reinterpret_cast<float*>(ws + L.q_scale);
+  auto k_scale = reinterpret_cast<float*>(ws + L.k_scale);
+  auto k_mean = reinterpret_cast<float*>(ws + L.k_mean);
+  auto v_scale = reinterpret_cast<float*>(ws + L.v_scale);
+  const PrepassScratch s = prepass_scratch_carve(ws + L.scratch, B * H, N, d);
+  cudaError_t e =
+      launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st);
+  if (e != cudaSuccess) return launch_status(e);
+  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
+                                        kDefaultTimeoutCycles, 0, st));
+}
+
+int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_fp, int8_t* modes_out) {
+  if (num_layers < 0 || n_fp < 0) return SAGE_EINVAL;
+  if (n_fp > 0 && !full_precision_layers) return SAGE_EINVAL;
+  if (num_layers > 0 && !modes_out) return SAGE_EINVAL;
+  for (int i = 0; i < n_fp; ++i)
+    if (full_precision_layers[i] < 0 || full_precision_layers[i] >= num_layers) return SAGE_EINVAL;
+  for (int l = 0; l < num_layers; ++l) modes_out[l] = (int8_t)SAGE_MODE_INT8_FP8;
+  for (int i = 0; i < n_fp; ++i) modes_out[full_precision_layers[i]] = (int8_t)SAGE_MODE_BF16;
+  return SAGE_OK;
+}
+
+int sage_status(void* workspace, void* stream) {
+  if (!workspace) return SAGE_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SAGE_ELAUNCH;
+  if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return SAGE_ELAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE_ELAUNCH;
+  if (word & kStatusTimeout) return SAGE_ETIMEOUT;
+  return word ? SAGE_ELAUNCH : SAGE_OK;
+}
+
+const char* sage_strerror(int code) {
+  switch (code) {
+    case SAGE_OK: return "ok";
+    case SAGE_EINVAL: return "invalid argument (size, null or misaligned pointer, mode)";
+    case SAGE_EUNSUPPORTED: return "unsupported (head dim must be 64 or 128; device must be sm_100)";
+    case SAGE_ELAUNCH: return "CUDA launch or runtime error";
+    case SAGE_EWORKSPACE: return "workspace too small";
+    case SAGE_ETIMEOUT: return "a bounded device-side wait ran out";
+    default: return "unknown status";
+  }
+}
+
+int sage_device_check(void) { return check_device(); }
+
+int sage_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int B, int H, int N, int d, const int* tile_list, int n,
+                      int32_t* out, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  if (n < 1 || n > 65535 || !q_i8 || !k_i8 || !tile_list || !out || !aligned16(q_i8) || !aligned16(k_i8))
+    return SAGE_EINVAL;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  return launch_status(
+      launch_dbg_qk_tiles(q_i8, k_i8, B * H, H, N, d, tile_list, n, out, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_dbg_pv_tile(const void* p, const void* vt, int d, int mode, float* out, void* stream) {
+  if (d != 64 && d != 128) return SAGE_EUNSUPPORTED;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8) return SAGE_EINVAL;
+  if (!p || !vt || !out || !aligned16(p) || !aligned16(vt)) return SAGE_EINVAL;
+  int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_dbg_pv_tile(p, vt, d, mode, out, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_dbg_qk_bf16_tile(const void* q, const void* k, int d, float* out, void* stream) {
+  if (d != 64 && d != 128) return SAGE_EUNSUPPORTED;
+  if (!q || !k || !out || !aligned16(q) || !aligned16(k)) return SAGE_EINVAL;
+  int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_dbg_qk_bf16_tile(q, k, d, out, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_dbg_attn_forced_timeout(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                                 const uint8_t* v_f8t, const float* v_scale, void* o, int B, int H, int N, int d,
+                                 void* status, long long timeout_cycles, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  const void* ptrs[] = {q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, status};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if (timeout_cycles < 1000 || timeout_cycles > kDefaultTimeoutCycles) return SAGE_EINVAL;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d,
+                                        static_cast<uint32_t*>(status), timeout_cycles, 1,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// internal.h -- declarations shared by the library's translation units (not
+// part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace sage {
+
+constexpr int kTile = 128;
+
+// Bits OR-ed into the device status word.
+constexpr uint32_t kStatusTimeout = 1u;
+
+inline int num_tiles(int N) { return (N + kTile - 1) / kTile; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Prepass scratch: per (bh, key block, channel) fp64 partial sums, fp32
+// block min / max of K and block absmax of V; per (bh, channel) V absmax.
+struct PrepassScratch {
+  double* k_psum;
+  float* k_pmin;
+  float* k_pmax;
+  float* v_pamax;
+  float* v_amax;
+};
+size_t prepass_scratch_bytes(int BH, int N, int d);
+PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d);
+
+cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
+                           float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
+                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream);
+
+// Quantized attention (INT8 QK^T, FP8 PV).  status: device uint32 word.
+cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                             const uint8_t* v_f8t, const float* v_scale, void* o, int BH, int N, int d,
+                             uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream);
+
+// BF16 attention.
+cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N, int d,
+                             uint32_t* status, long long timeout_cycles, cudaStream_t stream);
+
+// Diagnostics.
+cudaError_t launch_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int BH, int H, int N, int d,
+                                const int* tile_list, int n, int32_t* out, cudaStream_t stream);
+cudaError_t launch_dbg_pv_tile(const void* p, const void* vt, int d, int mode, float* out, cudaStream_t stream);
+cudaError_t launch_dbg_qk_bf16_tile(const void* q, const void* k, int d, float* out, cudaStream_t stream);
+
+// Tensor-map encoding through the driver entry point (no libcuda link).
+bool encode_tmap_2d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle);
+bool encode_tmap_3d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                    uint32_t box2, CUtensorMapSwizzle swizzle);
+
+// Default wait limit of the bounded device waits, in SM clocks (~1-2 s).
+constexpr long long kDefaultTimeoutCycles = 2000000000LL;
+
+}  // namespace sage

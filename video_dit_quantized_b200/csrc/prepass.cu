@@ -1,0 +1,299 @@
+// prepass.cu -- the quantization prepass of the SageAttention-style scheme
+// (page 1 of the TMAP write-up, "Attention performance optimisation":
+// SageAttention operator; zero-channel fix under "operator details").
+//
+// Three HBM-bound kernels, one CTA per (128-token block, head) where a block
+// is involved:
+//   stats     : Q block -> absmax -> INT8 codes + q_scale (single pass);
+//               K block -> per-channel fp64 partial sums (ascending tokens),
+//               fp32 min / max;  V block -> per-channel absmax.
+//   finalize  : per head, k_mean = fp32(sum of partials in ascending block
+//               order / N) and v_scale = amax / 448.
+//   quant_kv  : K block -> k_scale from (min, max, mean), smoothed INT8 codes;
+//               V block -> e4m3 codes of V * (448 / amax), written transposed.
+// All roundings are explicit (__f*_rn, cvt.rni, cvt.rn.satfinite) so that the
+// results are bit-for-bit those of the scheme's definition.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
+  x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x);
+  x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+  x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z);
+  x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ int quant_i8(float x, float inv) {
+  int c = __float2int_rn(__fmul_rn(x, inv));
+  return max(-127, min(127, c));
+}
+
+__device__ __forceinline__ uint2 pack_i8x8(const int (&c)[8]) {
+  uint2 r;
+  r.x = (uint32_t)(c[0] & 0xFF) | ((uint32_t)(c[1] & 0xFF) << 8) | ((uint32_t)(c[2] & 0xFF) << 16) |
+        ((uint32_t)(c[3] & 0xFF) << 24);
+  r.y = (uint32_t)(c[4] & 0xFF) | ((uint32_t)(c[5] & 0xFF) << 8) | ((uint32_t)(c[6] & 0xFF) << 16) |
+        ((uint32_t)(c[7] & 0xFF) << 24);
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+// grid (nK, BH)
+template <int D>
+__global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __restrict__ q,
+                                                                 const uint4* __restrict__ k,
+                                                                 const uint4* __restrict__ v, int N, int Npad,
+                                                                 int8_t* __restrict__ q_i8,
+                                                                 float* __restrict__ q_scale, PrepassScratch scr) {
+  constexpr int V8 = D / 8;                        // uint4 per token row
+  constexpr int PER_T = kTile * V8 / kThreads;     // uint4 per thread per block
+  static_assert(kThreads % V8 == 0, "a thread must always see the same 8 channels");
+  __shared__ __align__(16) uint4 ks[kTile * V8];
+  __shared__ int vamax_s[D];                       // non-negative floats as int bits
+  __shared__ float red[kThreads / 32];
+
+  const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
+  const int n0 = kb * kTile;
+  const int nr = min(kTile, N - n0);
+  const size_t in_base = ((size_t)bh * N + n0) * V8;  // in uint4
+
+  if (threadIdx.x < D) vamax_s[threadIdx.x] = 0;
+
+  // ---- Q: absmax over the block, then INT8 codes (one read) ----
+  uint4 qv[PER_T];
+  float amax = 0.f;
+  float va[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // V absmax of this thread's 8 channels
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int e = threadIdx.x + i * kThreads;       // uint4 index within block
+    const int row = e / V8;
+    qv[i] = make_uint4(0, 0, 0, 0);
+    if (row < nr) {
+      qv[i] = q[in_base + e];
+      ks[e] = k[in_base + e];
+      float y[8];
+      unpack8(v[in_base + e], y);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) va[u] = fmaxf(va[u], fabsf(y[u]));
+    }
+    float x[8];
+    unpack8(qv[i], x);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[u]));
+  }
+  amax = block_max(amax, red);   // also orders the vamax_s initialisation and the K staging
+  {
+    const int c0 = (threadIdx.x % V8) * 8;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) atomicMax(&vamax_s[c0 + u], __float_as_int(va[u]));
+  }
+  const float qinv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+  if (threadIdx.x == 0) q_scale[(size_t)bh * nK + kb] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+  uint2* qo = reinterpret_cast<uint2*>(q_i8 + ((size_t)bh * Npad + n0) * D);
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int e = threadIdx.x + i * kThreads;
+    float x[8];
+    unpack8(qv[i], x);
+    int c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = qinv > 0.f ? quant_i8(x[u], qinv) : 0;
+    qo[e] = pack_i8x8(c);   // rows >= nr hold zeros (qv was zeroed)
+  }
+  __syncthreads();
+
+  // ---- K column statistics (thread per channel, ascending tokens) ----
+  const __nv_bfloat16* kh = reinterpret_cast<const __nv_bfloat16*>(ks);
+  const size_t pidx = ((size_t)bh * nK + kb) * D;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    double s = 0.0;
+    float mn = __bfloat162float(kh[c]), mx = mn;
+    for (int n = 0; n < nr; ++n) {
+      const float x = __bfloat162float(kh[n * D + c]);
+      s = __dadd_rn(s, (double)x);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    scr.k_psum[pidx + c] = s;
+    scr.k_pmin[pidx + c] = mn;
+    scr.k_pmax[pidx + c] = mx;
+    scr.v_pamax[pidx + c] = __int_as_float(vamax_s[c]);
+  }
+}
+
+// grid (BH), block D
+template <int D>
+__global__ void prepass_finalize_kernel(int N, int nK, PrepassScratch scr, float* __restrict__ k_mean,
+                                        float* __restrict__ v_scale) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  double total = 0.0;
+  float a = 0.f;
+  for (int t = 0; t < nK; ++t) {
+    const size_t idx = ((size_t)bh * nK + t) * D + c;
+    total = __dadd_rn(total, scr.k_psum[idx]);
+    a = fmaxf(a, scr.v_pamax[idx]);
+  }
+  k_mean[(size_t)bh * D + c] = __double2float_rn(__ddiv_rn(total, (double)N));
+  v_scale[(size_t)bh * D + c] = a > 0.f ? __fdiv_rn(a, 448.0f) : 0.f;
+  scr.v_amax[(size_t)bh * D + c] = a;
+}
+
+// grid (nK, BH)
+template <int D>
+__global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4* __restrict__ k,
+                                                                    const uint4* __restrict__ v, int N, int Npad,
+                                                                    const float* __restrict__ k_mean,
+                                                                    int8_t* __restrict__ k_i8,
+                                                                    float* __restrict__ k_scale,
+                                                                    uint8_t* __restrict__ v_f8t, PrepassScratch scr) {
+  constexpr int V8 = D / 8;
+  constexpr int PER_T = kTile * V8 / kThreads;
+  __shared__ float mean_s[D];
+  __shared__ float vinv_s[D];
+  __shared__ __align__(16) uint4 vs[kTile * V8];
+  __shared__ float red[kThreads / 32];
+
+  const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
+  const int n0 = kb * kTile;
+  const int nr = min(kTile, N - n0);
+  const size_t in_base = ((size_t)bh * N + n0) * V8;
+  const size_t pidx = ((size_t)bh * nK + kb) * D;
+
+  // k_scale of this block from the partial min / max: fp32 subtraction is
+  // monotone, so max|fl(x - m)| over the block is attained at its min or max.
+  float kam = 0.f;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    const float m = k_mean[(size_t)bh * D + c];
+    mean_s[c] = m;
+    kam = fmaxf(fabsf(__fsub_rn(scr.k_pmax[pidx + c], m)), fabsf(__fsub_rn(scr.k_pmin[pidx + c], m)));
+    const float a = scr.v_amax[(size_t)bh * D + c];
+    vinv_s[c] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
+  }
+  kam = block_max(kam, red);   // contains __syncthreads
+  const float kinv = kam > 0.f ? __fdiv_rn(127.0f, kam) : 0.f;
+  if (threadIdx.x == 0) k_scale[(size_t)bh * nK + kb] = kam > 0.f ? __fdiv_rn(kam, 127.0f) : 0.f;
+
+  // ---- K: smoothed INT8 codes ----
+  uint2* ko = reinterpret_cast<uint2*>(k_i8 + ((size_t)bh * Npad + n0) * D);
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int e = threadIdx.x + i * kThreads;
+    const int row = e / V8, c0 = (e % V8) * 8;
+    int c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (row < nr && kinv > 0.f) {
+      float x[8];
+      unpack8(k[in_base + e], x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
+    }
+    ko[e] = pack_i8x8(c);
+  }
+
+  // ---- V: stage the block, then e4m3 codes written channel-major ----
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int e = threadIdx.x + i * kThreads;
+    const int row = e / V8;
+    vs[e] = row < nr ? v[in_base + e] : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
+  const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(vs);
+  constexpr int PAIRS = D * (kTile / 16);   // (channel, 16-token chunk)
+#pragma unroll
+  for (int i = 0; i < PAIRS / kThreads; ++i) {
+    const int p = threadIdx.x + i * kThreads;
+    const int c = p % D, chunk = p / D;
+    const float inv = vinv_s[c];
+    uint32_t w[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int n = chunk * 16 + g * 4 + u;
+        x[u] = __fmul_rn(__bfloat162float(vh[n * D + c]), inv);
+      }
+      w[g] = inv > 0.f ? pack_e4m3x4(x[0], x[1], x[2], x[3]) : 0u;
+    }
+    // padding tokens (n >= nr) were staged as +0 and encode to 0x00
+    uint4* dst = reinterpret_cast<uint4*>(v_f8t + ((size_t)bh * D + c) * Npad + (size_t)n0 + chunk * 16);
+    *dst = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int D>
+cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH, int N, int8_t* q_i8,
+                             float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
+                             float* v_scale, const PrepassScratch& scr, cudaStream_t stream) {
+  const int nK = num_tiles(N), Npad = nK * kTile;
+  dim3 grid(nK, BH);
+  prepass_stats_kernel<D><<<grid, kThreads, 0, stream>>>(
+      static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
+      q_scale, scr);
+  prepass_finalize_kernel<D><<<BH, D, 0, stream>>>(N, nK, scr, k_mean, v_scale);
+  prepass_quant_kv_kernel<D><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(k),
+                                                            static_cast<const uint4*>(v), N, Npad, k_mean, k_i8,
+                                                            k_scale, v_f8t, scr);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t prepass_scratch_bytes(int BH, int N, int d) {
+  const size_t n = (size_t)BH * num_tiles(N) * d;
+  return align_up(n * 8, 256) + 3 * align_up(n * 4, 256) + align_up((size_t)BH * d * 4, 256);
+}
+
+PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d) {
+  const size_t n = (size_t)BH * num_tiles(N) * d;
+  char* p = static_cast<char*>(base);
+  PrepassScratch s;
+  s.k_psum = reinterpret_cast<double*>(p);
+  p += align_up(n * 8, 256);
+  s.k_pmin = reinterpret_cast<float*>(p);
+  p += align_up(n * 4, 256);
+  s.k_pmax = reinterpret_cast<float*>(p);
+  p += align_up(n * 4, 256);
+  s.v_pamax = reinterpret_cast<float*>(p);
+  p += align_up(n * 4, 256);
+  s.v_amax = reinterpret_cast<float*>(p);
+  return s;
+}
+
+cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
+                           float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
+                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream) {
+  if (d == 128)
+    return launch_prepass_d<128>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
+                                 stream);
+  if (d == 64)
+    return launch_prepass_d<64>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
+                                stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sage

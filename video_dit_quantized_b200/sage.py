@@ -1,0 +1,223 @@
+"""Thin ctypes binding of the sage C ABI (include/sage.h).
+
+Argument marshalling only: every step of the attention path runs in the
+CUDA kernels of libsage.so.  torch is used for device memory and streams.
+There is no fallback: if the library cannot be loaded, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+from . import build as _build
+
+MODE_BF16 = 0
+MODE_INT8_FP8 = 1
+BLK = 128
+P_SCALE = 448.0
+
+OK, EINVAL, EUNSUPPORTED, ELAUNCH, EWORKSPACE, ETIMEOUT = 0, -1, -2, -3, -4, -5
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sage.h")
+
+
+class SageError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libsage.so is not built ({path}); run video_dit_quantized_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
+    sig = {
+        "sage_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
+        "sage_prepass_scratch_bytes": (sz, [i32, i32, i32, i32]),
+        "sage_quantize_qk": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sage_attn_quantized": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
+        "sage_attn_fwd": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]),
+        "attn_layer_schedule": (i32, [i32, vp, i32, vp]),
+        "sage_status": (i32, [vp, vp]),
+        "sage_strerror": (ctypes.c_char_p, [i32]),
+        "sage_device_check": (i32, []),
+        "sage_dbg_qk_tiles": (i32, [vp, vp, i32, i32, i32, i32, vp, i32, vp, vp]),
+        "sage_dbg_pv_tile": (i32, [vp, vp, i32, i32, vp, vp]),
+        "sage_dbg_qk_bf16_tile": (i32, [vp, vp, i32, vp, vp]),
+        "sage_dbg_attn_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/sage.h."""
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", txt, flags=re.M)
+
+
+def strerror(code: int) -> str:
+    return LIB.sage_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise SageError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bhnd(t, name):
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, H, N, d]")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.shape
+
+
+def workspace_bytes(B: int, H: int, N: int, d: int, mode: int) -> int:
+    return int(LIB.sage_workspace_bytes(B, H, N, d, mode))
+
+
+def prepass_scratch_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(LIB.sage_prepass_scratch_bytes(B, H, N, d))
+
+
+def alloc_workspace(B: int, H: int, N: int, d: int, mode: int, device=None):
+    import torch
+    n = workspace_bytes(B, H, N, d, mode)
+    if n == 0:
+        raise SageError(EINVAL, "sage_workspace_bytes")
+    ws = torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+    return ws
+
+
+def quantize_qk(q, k, v, stream=None):
+    """Runs the prepass; returns a dict of device tensors (q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale)."""
+    import torch
+    B, H, N, d = _bhnd(q, "q")
+    dev = q.device
+    nT = (N + BLK - 1) // BLK
+    out = dict(
+        q_i8=torch.empty((B, H, nT * BLK, d), dtype=torch.int8, device=dev),
+        q_scale=torch.empty((B, H, nT), dtype=torch.float32, device=dev),
+        k_i8=torch.empty((B, H, nT * BLK, d), dtype=torch.int8, device=dev),
+        k_scale=torch.empty((B, H, nT), dtype=torch.float32, device=dev),
+        k_mean=torch.empty((B, H, d), dtype=torch.float32, device=dev),
+        v_f8t=torch.empty((B, H, d, nT * BLK), dtype=torch.uint8, device=dev),
+        v_scale=torch.empty((B, H, d), dtype=torch.float32, device=dev),
+    )
+    nscr = prepass_scratch_bytes(B, H, N, d)
+    scratch = torch.empty(max(nscr, 256), dtype=torch.uint8, device=dev)
+    _check(LIB.sage_quantize_qk(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(out["q_i8"]), _ptr(out["q_scale"]),
+                                _ptr(out["k_i8"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]), _ptr(out["v_f8t"]),
+                                _ptr(out["v_scale"]), _ptr(scratch), scratch.numel(), _stream(stream)),
+           "sage_quantize_qk")
+    out["_scratch"] = scratch
+    return out
+
+
+def attn_quantized(pre: dict, N: int, o=None, status=None, stream=None):
+    """Attention over prepass outputs; returns bf16 O [B,H,N,d]."""
+    import torch
+    B, H, _, d = pre["q_i8"].shape
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=pre["q_i8"].device)
+    if status is None:
+        status = torch.zeros(64, dtype=torch.int32, device=o.device)
+    _check(LIB.sage_attn_quantized(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]), _ptr(pre["k_scale"]),
+                                   _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o), B, H, N, d, _ptr(status),
+                                   _stream(stream)), "sage_attn_quantized")
+    return o
+
+
+def attn_fwd(q, k, v, mode: int, o=None, workspace=None, stream=None):
+    """Full-sequence self-attention through sage_attn_fwd; returns bf16 O [B,H,N,d]."""
+    import torch
+    B, H, N, d = _bhnd(q, "q")
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, mode, q.device)
+    _check(LIB.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(mode), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)), "sage_attn_fwd")
+    return o
+
+
+def status(workspace, stream=None) -> int:
+    """Reads and clears the device status word (synchronises the stream); returns a status code."""
+    return int(LIB.sage_status(_ptr(workspace), _stream(stream)))
+
+
+def layer_schedule(num_layers: int, full_precision_layers) -> list[int]:
+    """Per-layer modes: MODE_BF16 for the listed layers, MODE_INT8_FP8 for the rest (host only)."""
+    fp = list(full_precision_layers)
+    arr = (ctypes.c_int * max(len(fp), 1))(*fp)
+    modes = (ctypes.c_int8 * max(num_layers, 1))()
+    _check(LIB.attn_layer_schedule(int(num_layers), ctypes.cast(arr, ctypes.c_void_p), len(fp),
+                                   ctypes.cast(modes, ctypes.c_void_p)), "attn_layer_schedule")
+    return [int(modes[i]) for i in range(num_layers)]
+
+
+def device_check() -> int:
+    return int(LIB.sage_device_check())
+
+
+# ---------------------------------------------------------------- diagnostics
+
+def dbg_qk_tiles(q_i8, k_i8, N: int, tiles, stream=None):
+    """int32 QK^T tiles [(b,h,qb,kb)...] -> [n,128,128] through the tcgen05 kind::i8 path."""
+    import torch
+    B, H, _, d = q_i8.shape
+    tl = torch.tensor(tiles, dtype=torch.int32, device=q_i8.device).reshape(-1, 4).contiguous()
+    out = torch.empty((tl.shape[0], BLK, BLK), dtype=torch.int32, device=q_i8.device)
+    _check(LIB.sage_dbg_qk_tiles(_ptr(q_i8), _ptr(k_i8), B, H, N, d, _ptr(tl), tl.shape[0], _ptr(out),
+                                 _stream(stream)), "sage_dbg_qk_tiles")
+    return out
+
+
+def dbg_pv_tile(p, vt, mode: int, stream=None):
+    import torch
+    d = vt.shape[0] if mode == MODE_INT8_FP8 else vt.shape[1]
+    out = torch.empty((BLK, d), dtype=torch.float32, device=p.device)
+    _check(LIB.sage_dbg_pv_tile(_ptr(p), _ptr(vt), d, int(mode), _ptr(out), _stream(stream)), "sage_dbg_pv_tile")
+    return out
+
+
+def dbg_qk_bf16_tile(q, k, stream=None):
+    import torch
+    d = q.shape[1]
+    out = torch.empty((BLK, BLK), dtype=torch.float32, device=q.device)
+    _check(LIB.sage_dbg_qk_bf16_tile(_ptr(q), _ptr(k), d, _ptr(out), _stream(stream)), "sage_dbg_qk_bf16_tile")
+    return out
+
+
+def dbg_attn_forced_timeout(pre: dict, N: int, status, timeout_cycles: int, o=None, stream=None):
+    import torch
+    B, H, _, d = pre["q_i8"].shape
+    if o is None:
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=pre["q_i8"].device)
+    _check(LIB.sage_dbg_attn_forced_timeout(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]),
+                                            _ptr(pre["k_scale"]), _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o),
+                                            B, H, N, d, _ptr(status), int(timeout_cycles), _stream(stream)),
+           "sage_dbg_attn_forced_timeout")
+    return o
