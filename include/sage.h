@@ -17,7 +17,8 @@
  *    B * H * ceil(N/128) * 128 * d < 2^31.
  *  - Pointers are DEVICE pointers unless a parameter says "host".  Device
  *    pointers must be 16-byte aligned.  The caller owns all memory; the
- *    library allocates nothing and keeps no state between calls.
+ *    library allocates nothing and keeps no state between calls, except the
+ *    fixed scratch array of sage_quantize_qk_noalloc (see there).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Calls are asynchronous on that stream; no call synchronises except
  *    sage_status().
@@ -90,6 +91,33 @@ int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, 
                      int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
                      uint8_t* v_f8t, float* v_scale, void* scratch, size_t scratch_bytes,
                      void* stream);
+
+/*
+ * Same prepass as sage_quantize_qk, for callers that must not allocate device
+ * memory while they run (a service that reserved all of HBM for its own pool,
+ * a latency-critical loop that cannot take the implicit synchronisation of
+ * cudaMalloc / cudaFree).  The pages this library follows describe no such
+ * entry point; it exists for those callers only.
+ *  - The prepass partials live in one fixed device array inside the library,
+ *    SAGE_NOALLOC_SCRATCH_BYTES (32 MiB) on every device that loads it, held
+ *    until the process exits.  The caller passes only inputs and outputs
+ *    (same meaning and layout as sage_quantize_qk).
+ *  - Problems whose partials need more than that (sage_prepass_scratch_bytes
+ *    > SAGE_NOALLOC_SCRATCH_BYTES, e.g. B*H*ceil(N/128)*d above ~1.6M) are
+ *    rejected with SAGE_EWORKSPACE before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device, with that device current); make
+ *    that first call before any stream capture.
+ *  - Every call shares the one array.  Calls whose kernels may overlap on the
+ *    GPU (different streams, or several host threads) race on it and give
+ *    wrong results: serialise them on one stream.  Each call overwrites every
+ *    partial it later reads, so no clearing is needed between calls.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define SAGE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int sage_quantize_qk_noalloc(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                             int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                             uint8_t* v_f8t, float* v_scale, void* stream);
 
 /*
  * Attention over already-quantized operands (steps a5-a9): per 128x128 tile

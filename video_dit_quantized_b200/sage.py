@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
         "sage_dbg_pv_tile": (i32, [vp, vp, i32, i32, vp, vp]),
         "sage_dbg_qk_bf16_tile": (i32, [vp, vp, i32, vp, vp]),
         "sage_dbg_attn_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
+        "sage_quantize_qk_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -134,6 +135,21 @@ def quantize_qk(q, k, v, stream=None):
            "sage_quantize_qk")
     out["_scratch"] = scratch
     return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def quantize_qk_noalloc(q, k, v, out: dict, stream=None) -> int:
+    """The prepass through sage_quantize_qk_noalloc: its scratch is the library's
+    fixed device array, so the call itself allocates nothing.  `out` holds
+    caller-allocated outputs with the keys and shapes quantize_qk returns.
+    Returns the status code (SAGE_EWORKSPACE if the problem exceeds the array)."""
+    B, H, N, d = _bhnd(q, "q")
+    return int(LIB.sage_quantize_qk_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(out["q_i8"]),
+                                            _ptr(out["q_scale"]), _ptr(out["k_i8"]), _ptr(out["k_scale"]),
+                                            _ptr(out["k_mean"]), _ptr(out["v_f8t"]), _ptr(out["v_scale"]),
+                                            _stream(stream)))
 
 
 def attn_quantized(pre: dict, N: int, o=None, status=None, stream=None):
