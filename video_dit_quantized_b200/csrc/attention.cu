@@ -4,27 +4,31 @@
 // on page 1 of the TMAP write-up ("Attention performance optimisation /
 // Background") and replaced there by the SageAttention operator ("attention
 // quantization"), with some layers kept at original precision ("keeping
-// video quality").  Two instantiations of one pipeline:
+// video quality").  Two instantiations of one warp-specialised pipeline:
 //   QUANT = true : S = Q_i8 K_i8^T (tcgen05 kind::i8, exact int32), dequant
 //                  with q_scale * k_scale * log2(e)/sqrt(d), P8 = e4m3(p*448)
-//                  kept in tensor memory, O += P8 V8 (kind::f8f6f4, fp32).
+//                  staged in shared memory, O += P8 V8 (kind::f8f6f4, fp32).
 //   QUANT = false: S = Q K^T and O += P V with kind::f16 (bf16 in, fp32 acc),
-//                  P rounded to bf16 in tensor memory.
+//                  P rounded to bf16 and kept in tensor memory over S.
 //
 // One CTA = two 128-row Q tiles of one (b, h) and every 128-key tile of that
-// head.  Warp roles (12 warps):
+// head.  Warp roles (12 warps, registers re-split with setmaxnreg):
 //   warp 0      TMA producer: Q tiles once, then K/V tiles through a ring of
 //               STAGES shared-memory slots (mbarrier full / empty pairs);
 //   warp 1      TMEM allocator and the single MMA-issuing thread;
 //   warps 4-7   softmax for Q tile 0, warps 8-11 for Q tile 1: one thread
-//               per query row (TMEM lane), online softmax in registers, P
-//               written back over its S columns, O rescaled in place, and the
-//               epilogue (normalise, round to bf16, store).
+//               per query row (TMEM lane), online softmax in registers, O
+//               rescaled in place in TMEM, and the epilogue.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
-// Per key tile j the MMA thread issues PV_t(j) and then QK_t(j+1) into the
-// same S_t columns; tcgen05 operations from one thread execute in order, and
-// the commit after QK_t(j+1) also covers PV_t(j), so when the softmax warps
-// see S_t(j+1) the accumulator O_t is stable and may be rescaled.
+//
+// QUANT schedule: as soon as a softmax warpgroup has S_t(j) in registers it
+// releases the S columns (s_free), so the MMA thread issues QK_t(j+1) while
+// the exponentials of step j run; P_t(j) goes to shared memory and PV_t(j)
+// (an SS MMA) is issued on p_full.  The commit after PV_t(j) (o_ready) tells
+// the warpgroup that O_t is stable and the P buffer is free again.
+// BF16 schedule: P_t(j) overwrites S_t(j) in TMEM, so QK_t(j+1) follows PV_t(j)
+// in issue order; tcgen05 operations from one thread execute in order and the
+// commit after QK_t(j+1) also covers PV_t(j), so S_t(j+1) implies O_t stable.
 //
 // Every wait is bounded (clock64 limit); a wait that runs out raises a
 // CTA-wide abort flag, every role leaves its loop, in-flight TMA loads and
@@ -44,6 +48,10 @@ namespace {
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kTmemCols = 512;
+// Register split: the kernel is compiled for kLaunchRegs per thread (384 threads,
+// one CTA per SM); warpgroup 0 (producer, MMA, idle warps) drops to Cfg::REGS_LOW
+// and the two softmax warpgroups rise to Cfg::REGS_HIGH, within 384 * 168.
+constexpr int kLaunchRegs = 168;
 
 // log2(e) / sqrt(d), formed in double and rounded once to fp32
 __host__ __device__ constexpr float softmax_c(int d) {
@@ -55,11 +63,13 @@ template <int D, bool QUANT>
 struct Cfg {
   static constexpr int ELEM = QUANT ? 1 : 2;
   static constexpr int TILE_BYTES = 128 * D * ELEM;               // one Q, K or V tile
+  static constexpr int P_BYTES = QUANT ? 128 * 128 : 0;           // one e4m3 P tile in smem
   static constexpr int STAGES = QUANT ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 3);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;          // barriers + 1 KB alignment slack
   // Q/K operand rows in shared memory (bytes) and their swizzle
   static constexpr int QK_ROW = QUANT ? D : 128;                   // bf16: one 64-element atom
@@ -67,13 +77,15 @@ struct Cfg {
   static constexpr uint32_t QK_SBO = 8 * QK_ROW;
   static constexpr int QK_KSTEPS = QUANT ? D / 32 : D / 16;
   static constexpr int PV_KSTEPS = QUANT ? 128 / 32 : 128 / 16;
-  static constexpr int P_COLS = QUANT ? 32 : 64;                   // TMEM columns of P per row
   static constexpr uint32_t IDESC_QK =
       QUANT ? make_idesc(kFmtS32Acc, kFmtS8, kFmtS8, 0, 128, 128) : make_idesc(kFmtF32Acc, kFmtBF16, kFmtBF16, 0, 128, 128);
   static constexpr uint32_t IDESC_PV =
       QUANT ? make_idesc(kFmtF32Acc, kFmtE4M3, kFmtE4M3, 0, 128, D) : make_idesc(kFmtF32Acc, kFmtBF16, kFmtBF16, 1, 128, D);
   static constexpr int KIND_QK = QUANT ? kKindI8 : kKindF16;
-  static constexpr int KIND_PV = QUANT ? kKindF8F6F4 : kKindF16;
+  static constexpr int REGS_LOW = QUANT ? 96 : 80;
+  static constexpr int REGS_HIGH = QUANT ? 200 : 208;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // S[tmem] = Q[smem] K[smem]^T for one 128x128 tile (K-major operands).
@@ -90,21 +102,40 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
   }
 }
 
-// O[tmem] (+)= P[tmem] V[smem] for one 128-key tile.
-//  QUANT: V^T tile [D rows][128 keys] e4m3, K-major, 128-byte swizzle.
-//  bf16 : V tile [128 keys][D] as 64-channel atoms (16 KB each), MN-major.
-template <int D, bool QUANT>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t accumulate) {
-  using C = Cfg<D, QUANT>;
+// QUANT: O[tmem] (+)= P8[smem] V8[smem] for one 128-key tile.  P tile [128 rows]
+// [128 keys] e4m3 and V^T tile [D rows][128 keys] e4m3, both K-major with the
+// 128-byte swizzle; 32-byte K steps.
+template <int D>
+__device__ __forceinline__ void issue_pv_quant(uint32_t d_tmem, uint32_t p_smem, uint32_t v_smem, uint32_t accumulate) {
+  using C = Cfg<D, true>;
 #pragma unroll
   for (int s = 0; s < C::PV_KSTEPS; ++s) {
-    uint64_t b;
-    if constexpr (QUANT)
-      b = make_sdesc(v_smem + s * 32, 16, 1024, kLayoutSW128);
-    else
-      b = make_sdesc(v_smem + s * 2048, 16384, 1024, kLayoutSW128);
-    mma_ts<C::KIND_PV>(d_tmem, p_tmem + s * 8, b, C::IDESC_PV, (s > 0 || accumulate) ? 1u : 0u);
+    const uint64_t a = make_sdesc(p_smem + s * 32, 16, 1024, kLayoutSW128);
+    const uint64_t b = make_sdesc(v_smem + s * 32, 16, 1024, kLayoutSW128);
+    mma_ss<kKindF8F6F4>(d_tmem, a, b, C::IDESC_PV, (s > 0 || accumulate) ? 1u : 0u);
   }
+}
+
+// BF16: O[tmem] (+)= P[tmem] V[smem]; V tile [128 keys][D] stored as 64-channel
+// atoms (16 KB each), MN-major; P bf16 in TMEM (64 columns).
+template <int D>
+__device__ __forceinline__ void issue_pv_bf16(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t accumulate) {
+  using C = Cfg<D, false>;
+#pragma unroll
+  for (int s = 0; s < C::PV_KSTEPS; ++s) {
+    const uint64_t b = make_sdesc(v_smem + s * 2048, 16384, 1024, kLayoutSW128);
+    mma_ts<kKindF16>(d_tmem, p_tmem + s * 8, b, C::IDESC_PV, (s > 0 || accumulate) ? 1u : 0u);
+  }
+}
+
+// One thread's 128-byte P row into a [128 x 128 B] tile with the 128-byte
+// swizzle (16-byte chunk c of row r sits at chunk position c ^ (r % 8)); the
+// tile base is 1024-byte aligned.
+__device__ __forceinline__ void store_p_row(uint8_t* tile, int row, const uint32_t (&pk)[32]) {
+  uint8_t* rp = tile + row * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
 }
 
 struct Params {
@@ -130,10 +161,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;                       // [STAGES]
   uint64_t* kv_empty = bars + 1 + C::STAGES;          // [STAGES]
-  uint64_t* s_full = bars + 1 + 2 * C::STAGES;        // [2]
-  uint64_t* p_full = s_full + 2;                      // [2]
-  uint64_t* o_final = p_full + 2;                     // [2]
-  uint64_t* mma_done = o_final + 2;
+  uint64_t* s_full = bars + 1 + 2 * C::STAGES;        // [2] S_t written (MMA commit)
+  uint64_t* s_free = s_full + 2;                      // [2] S_t read into registers (QUANT)
+  uint64_t* p_full = s_free + 2;                      // [2] P_t written, O_t rescaled
+  uint64_t* o_ready = p_full + 2;                     // [2] PV_t done (QUANT: every step; BF16: last)
+  uint64_t* tok = o_ready + 2;                        // [2] exp-phase token of softmax warpgroup t
+  uint64_t* mma_done = tok + 2;
   uint64_t* never = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -152,8 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
       mbar_init(&p_full[t], 128);
-      mbar_init(&o_final[t], 1);
+      mbar_init(&o_ready[t], 1);
+      mbar_init(&tok[t], 128);
     }
     mbar_init(mma_done, 1);
     mbar_init(never, 1);
@@ -169,9 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < 4) {
+    regs_release<C::REGS_LOW>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- producer
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -209,13 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(q_full, 0, &no_abort, limit);
       for (int j = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; j < issued; ++j)
         mbar_wait(&kv_full[j % C::STAGES], (j / C::STAGES) & 1, &no_abort, limit);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t q_s = smem_u32(smem + C::OFF_Q);
       const uint32_t k_s = smem_u32(smem + C::OFF_K);
       const uint32_t v_s = smem_u32(smem + C::OFF_V);
+      const uint32_t p_s = smem_u32(smem + C::OFF_P);
       bool ok = true;
       if (prm.dbg_flags & 1) ok = mbar_wait(never, 0, abort_flag, limit);
       ok = ok && mbar_wait(q_full, 0, abort_flag, limit) && mbar_wait(&kv_full[0], 0, abort_flag, limit);
@@ -225,25 +260,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_qk<D, QUANT>(tmem + t * 128, q_s + t * C::TILE_BYTES, k_s);
           mma_commit(&s_full[t]);
         }
+        if constexpr (QUANT) {
+          // Event driven: each tile runs QK(1), PV(0), QK(2), PV(1), ... as its
+          // barriers allow, so one slow tile never holds back the other.
+          //   QK_t(j+1) needs s_free_t(j) (S_t(j) read out) and K_{j+1} loaded;
+          //   PV_t(j)   needs p_full_t(j) (P_t(j) stored, O_t rescaled).
+          int qk_next[2] = {1, 1}, pv_next[2] = {0, 0};
+          long long last = clock64();
+          while (ok && (pv_next[0] < nT || pv_next[1] < nT)) {
+            bool progressed = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int jq = qk_next[t];
+              if (jq < nT && mbar_test(&s_free[t], (jq - 1) & 1) &&
+                  mbar_test(&kv_full[jq % C::STAGES], (jq / C::STAGES) & 1)) {
+                tc_fence_after();
+                issue_qk<D, true>(tmem + t * 128, q_s + t * C::TILE_BYTES, k_s + (jq % C::STAGES) * C::TILE_BYTES);
+                mma_commit(&s_full[t]);
+                qk_next[t] = jq + 1;
+                progressed = true;
+              }
+              const int jp = pv_next[t];
+              if (jp < qk_next[t] && jp < nT && mbar_test(&p_full[t], jp & 1)) {
+                tc_fence_after();
+                issue_pv_quant<D>(tmem + 256 + t * D, p_s + t * C::P_BYTES, v_s + (jp % C::STAGES) * C::TILE_BYTES,
+                                  jp > 0 ? 1u : 0u);
+                mma_commit(&o_ready[t]);
+                pv_next[t] = jp + 1;
+                // the K/V stage of step jp is free once both tiles' PV(jp) are issued
+                if (pv_next[1 - t] > jp) mma_commit(&kv_empty[jp % C::STAGES]);
+                progressed = true;
+              }
+            }
+            if (progressed) {
+              last = clock64();
+            } else if (*abort_flag || clock64() - last > limit) {
+              *abort_flag = 1;
+              ok = false;
+            } else {
+              __nanosleep(20);   // leave the issue slots to the softmax warps on this SMSP
+            }
+          }
+        } else {
         for (int j = 0; j < nT && ok; ++j) {
           const int s = j % C::STAGES;
-          for (int t = 0; t < 2; ++t) {
-            if (!mbar_wait(&p_full[t], j & 1, abort_flag, limit)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv<D, QUANT>(tmem + 256 + t * D, tmem + t * 128, v_s + s * C::TILE_BYTES, j > 0 ? 1u : 0u);
-            if (j + 1 < nT) {
-              const int s1 = (j + 1) % C::STAGES;
-              if (t == 0 && !mbar_wait(&kv_full[s1], ((j + 1) / C::STAGES) & 1, abort_flag, limit)) {
-                ok = false;
-                break;
+          {
+            for (int t = 0; t < 2; ++t) {
+              if (!mbar_wait(&p_full[t], j & 1, abort_flag, limit)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv_bf16<D>(tmem + 256 + t * D, tmem + t * 128, v_s + s * C::TILE_BYTES, j > 0 ? 1u : 0u);
+              if (j + 1 < nT) {
+                const int s1 = (j + 1) % C::STAGES;
+                if (t == 0 && !mbar_wait(&kv_full[s1], ((j + 1) / C::STAGES) & 1, abort_flag, limit)) {
+                  ok = false;
+                  break;
+                }
+                issue_qk<D, false>(tmem + t * 128, q_s + t * C::TILE_BYTES, k_s + s1 * C::TILE_BYTES);
+                mma_commit(&s_full[t]);
+              } else {
+                mma_commit(&o_ready[t]);
               }
-              issue_qk<D, QUANT>(tmem + t * 128, q_s + t * C::TILE_BYTES, k_s + s1 * C::TILE_BYTES);
-              mma_commit(&s_full[t]);
-            } else {
-              mma_commit(&o_final[t]);
             }
           }
           if (ok) mma_commit(&kv_empty[s]);
+        }
         }
       }
       // drain: every MMA issued must complete before TMEM is released
@@ -251,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int no_abort = 0;
       mbar_wait(mma_done, 0, &no_abort, limit);
     }
-  } else if (warp >= 4) {
+  } else {
+    regs_claim<C::REGS_HIGH>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
@@ -259,104 +340,161 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * D;
+    uint8_t* p_tile = smem + C::OFF_P + t * C::P_BYTES;
     const int qt = qt0 + t;
     const float c = softmax_c(D);
     float qs = 1.0f;
     if constexpr (QUANT) qs = qt < nT ? prm.q_scale[(size_t)bh * nT + qt] : 0.f;
+    // QUANT: p is produced already multiplied by the P scale 448 (2^(s - m + log2 448)),
+    // so l accumulates 448 * sum(p) and the epilogue divides by it directly.
+    constexpr float kLog2PScale = QUANT ? 8.807354922057604f : 0.f;
+    // QUANT scores arrive as int32 S; S + 0x4B400000 read as a float is 12582912 + S
+    // exactly (|S| <= 127*127*128 < 2^22), a conversion on the integer ALU.
+    constexpr uint32_t kMagicBits = 0x4B400000u;
+    constexpr float kMagic = 12582912.0f;
+    float ks_next = 0.f;
+    if constexpr (QUANT) ks_next = prm.k_scale[(size_t)bh * nT];
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nT; ++j) {
+      float sc = c;
+      if constexpr (QUANT) {
+        sc = __fmul_rn(__fmul_rn(qs, ks_next), c);
+        if (j + 1 < nT) ks_next = prm.k_scale[(size_t)bh * nT + j + 1];   // prefetch the next tile's scale
+      }
       if (!mbar_wait(&s_full[t], j & 1, abort_flag, limit)) { ok = false; break; }
       tc_fence_after();
       const int valid = min(128, N - j * 128);
-      float sc = c;
-      if constexpr (QUANT) sc = __fmul_rn(__fmul_rn(qs, prm.k_scale[(size_t)bh * nT + j]), c);
-      // pass 1: row max of the raw scores (monotone in s since sc >= 0)
-      float mt;
+      // the whole S row in registers (one wait for four loads)
+      uint32_t sr[128];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32(tS + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[ch * 32]));
+      tmem_wait_ld();
       if constexpr (QUANT) {
-        int mx = INT_MIN;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(tS + ch * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < valid) mx = max(mx, (int)r[i]);
-        }
-        mt = __fmul_rn((float)mx, sc);
-      } else {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(tS + ch * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(r[i]));
-        }
-        mt = __fmul_rn(mx, sc);
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);     // the S columns may now take QK_t(j+1)
       }
-      const float m_new = fmaxf(m, mt);
+      // scores as floats: QUANT keeps 12582912 + S (exact) until after the max
+      float f[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) f[i] = QUANT ? __uint_as_float(sr[i] + kMagicBits) : __uint_as_float(sr[i]);
+      const bool full = valid == 128;
+      // row max of the raw scores (s is monotone in f since sc >= 0)
+      float mx;
+      if (full) {
+        float a0 = f[0], a1 = f[1], a2 = f[2], a3 = f[3];
+#pragma unroll
+        for (int i = 4; i < 128; i += 8) {
+          a0 = fmax3(a0, f[i], f[i + 1]);
+          a1 = fmax3(a1, f[i + 2], f[i + 3]);
+          a2 = fmax3(a2, f[i + 4], f[i + 5]);
+          a3 = fmax3(a3, f[i + 6], f[i + 7]);
+        }
+        mx = fmaxf(fmax3(a0, a1, a2), a3);
+      } else {
+        mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, i < valid ? f[i] : -INFINITY);
+      }
+      if constexpr (QUANT) {
+        mx = __fsub_rn(mx, kMagic);                       // exact: the integer max as a float
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) {                // exact: back to S as a float
+          const float2 v = fadd2(make_float2(f[i], f[i + 1]), make_float2(-kMagic, -kMagic));
+          f[i] = v.x;
+          f[i + 1] = v.y;
+        }
+      }
+      const float m_new = fmaxf(m, __fmul_rn(mx, sc));
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(__fsub_rn(m, m_new));
-      // rescale O_t (complete: the commit that signalled S_t(j) covers PV_t(j-1))
-      if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
+      const float bias = __fsub_rn(kLog2PScale, m_new);  // x = f * sc + bias = s - m_new (+ log2 448)
+      // The two warpgroups take turns on the exponential phase (the SFU-bound
+      // part), so each one's integer/compare phase overlaps the other's
+      // exponentials: warpgroup 0 goes first, then they alternate.
+      if (t == 1 || j > 0) {
+        if (!mbar_wait(&tok[t], (t == 0 ? (j - 1) : j) & 1, abort_flag, limit)) { ok = false; break; }
+      }
+      // p = 2^x, row sum (two packed accumulators), P packed for the PV MMA
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      uint32_t pk[QUANT ? 32 : 64];
+      if (full) {
+#pragma unroll
+        for (int g = 0; g < 32; ++g) {
+          const float2 x01 = ffma2(f[4 * g], f[4 * g + 1], sc, bias);
+          const float2 x23 = ffma2(f[4 * g + 2], f[4 * g + 3], sc, bias);
+          const float p0 = ex2_approx(x01.x), p1 = ex2_approx(x01.y), p2 = ex2_approx(x23.x), p3 = ex2_approx(x23.y);
+          acc0 = fadd2(acc0, make_float2(p0, p1));
+          acc1 = fadd2(acc1, make_float2(p2, p3));
+          if constexpr (QUANT) {
+            pk[g] = pack_e4m3x4(p0, p1, p2, p3);
+          } else {
+            pk[2 * g] = pack_bf16x2(p0, p1);
+            pk[2 * g + 1] = pack_bf16x2(p2, p3);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 32; ++g) {
+          const float2 x01 = ffma2(f[4 * g], f[4 * g + 1], sc, bias);
+          const float2 x23 = ffma2(f[4 * g + 2], f[4 * g + 3], sc, bias);
+          const float p0 = 4 * g + 0 < valid ? ex2_approx(x01.x) : 0.f;
+          const float p1 = 4 * g + 1 < valid ? ex2_approx(x01.y) : 0.f;
+          const float p2 = 4 * g + 2 < valid ? ex2_approx(x23.x) : 0.f;
+          const float p3 = 4 * g + 3 < valid ? ex2_approx(x23.y) : 0.f;
+          acc0 = fadd2(acc0, make_float2(p0, p1));
+          acc1 = fadd2(acc1, make_float2(p2, p3));
+          if constexpr (QUANT) {
+            pk[g] = pack_e4m3x4(p0, p1, p2, p3);
+          } else {
+            pk[2 * g] = pack_bf16x2(p0, p1);
+            pk[2 * g + 1] = pack_bf16x2(p2, p3);
+          }
+        }
+      }
+      mbar_arrive(&tok[1 - t]);     // hand the exponential phase to the other warpgroup
+      const bool grew = j > 0 && __any_sync(0xffffffffu, m_new > m);
+      if constexpr (QUANT) {
+        // PV_t(j-1) must be done: it reads the P buffer and updates O_t
+        if (j > 0) {
+          if (!mbar_wait(&o_ready[t], (j - 1) & 1, abort_flag, limit)) { ok = false; break; }
+          tc_fence_after();
+        }
+        store_p_row(p_tile, row, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        fence_proxy_async_smem();    // generic-proxy writes -> visible to the MMA
+      } else {
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      }
+      // rescale O_t by alpha where the max grew (O_t is complete: QUANT waited
+      // for o_ready above; BF16's S_t(j) commit covers PV_t(j-1))
+      if (grew) {
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(tO + ch * 32, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), alpha));
+          for (int i = 0; i < 32; i += 2) {
+            const float2 v = fmul2(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), alpha);
+            r[i] = __float_as_uint(v.x);
+            r[i + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(tO + ch * 32, r);
-        }
-        tmem_wait_st();
-      }
-      // pass 2: p = 2^(s - m_new), row sum, P written over the S columns
-      float psum = 0.f;
-      uint32_t pk[2 * 32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tS + ch * 32, r);
-        tmem_wait_ld();
-        float p[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float s = QUANT ? __fmul_rn((float)(int)r[i], sc) : __fmul_rn(__uint_as_float(r[i]), sc);
-          p[i] = (ch * 32 + i < valid) ? ex2_approx(__fsub_rn(s, m_new)) : 0.f;
-          psum = __fadd_rn(psum, p[i]);
-        }
-        if constexpr (QUANT) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g)
-            pk[ch * 8 + g] = pack_e4m3x4(__fmul_rn(p[4 * g], 448.f), __fmul_rn(p[4 * g + 1], 448.f),
-                                         __fmul_rn(p[4 * g + 2], 448.f), __fmul_rn(p[4 * g + 3], 448.f));
-        } else {
-#pragma unroll
-          for (int g = 0; g < 16; ++g) pk[ch * 16 + g] = pack_bf16x2(p[2 * g], p[2 * g + 1]);
-        }
-      }
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        tmem_st32(tS, lo);
-        if constexpr (!QUANT) {
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-          tmem_st32(tS + 32, hi);
         }
       }
       tmem_wait_st();
-      l = __fadd_rn(__fmul_rn(l, alpha), psum);
+      const float2 acc = fadd2(acc0, acc1);
+      l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(acc.x, acc.y));
       m = m_new;
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && mbar_wait(&o_final[t], 0, abort_flag, limit)) {
+    const uint32_t last_parity = QUANT ? (uint32_t)((nT - 1) & 1) : 0u;
+    if (ok && mbar_wait(&o_ready[t], last_parity, abort_flag, limit)) {
       tc_fence_after();
       const int gq = qt * 128 + row;
-      const float denom = QUANT ? __fmul_rn(448.f, l) : l;
+      const float denom = l;   // QUANT: l already holds 448 * sum(p)
       __nv_bfloat16* orow = prm.o + ((size_t)bh * N + gq) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -446,14 +584,18 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
-// One 128-row P.V product: P from global into TMEM (tcgen05.st), V via TMA.
+// One 128-row P.V product through the attention kernels' operand paths: QUANT
+// writes P rows into a swizzled shared-memory tile (store_p_row) and issues the
+// SS kind::f8f6f4 MMA; BF16 writes P into TMEM (tcgen05.st) and issues the TS
+// kind::f16 MMA with an MN-major V.  V arrives by TMA.
 template <int D, bool QUANT>
 __global__ void __launch_bounds__(128, 1)
     dbg_pv_kernel(const __grid_constant__ CUtensorMap tmV, const uint8_t* p, float* out) {
   using C = Cfg<D, QUANT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::TILE_BYTES);
+  uint8_t* p_tile = smem + C::TILE_BYTES;                           // QUANT only: [128 x 128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::TILE_BYTES + (QUANT ? 128 * 128 : 0));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   __shared__ int abort_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -473,14 +615,20 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const int row = warp * 32 + lane;
-  // P row -> TMEM columns [0, P_COLS) (P occupies the start of an S region)
   const uint32_t* prow = reinterpret_cast<const uint32_t*>(p + (size_t)row * 128 * (QUANT ? 1 : 2));
-  for (int h = 0; h < C::P_COLS / 32; ++h) {
+  if constexpr (QUANT) {
     uint32_t r[32];
-    for (int i = 0; i < 32; ++i) r[i] = prow[h * 32 + i];
-    tmem_st32(tmem + lane_off + h * 32, r);
+    for (int i = 0; i < 32; ++i) r[i] = prow[i];
+    store_p_row(p_tile, row, r);
+    fence_proxy_async_smem();
+  } else {
+    for (int h = 0; h < 2; ++h) {
+      uint32_t r[32];
+      for (int i = 0; i < 32; ++i) r[i] = prow[h * 32 + i];
+      tmem_st32(tmem + lane_off + h * 32, r);
+    }
+    tmem_wait_st();
   }
-  tmem_wait_st();
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -491,8 +639,12 @@ __global__ void __launch_bounds__(128, 1)
     } else {
       for (int a = 0; a < D / 64; ++a) tma_load_2d(smem + a * 16384, &tmV, &bars[0], a * 64, 0);
     }
-    if (mbar_wait(&bars[0], 0, &abort_s, kDefaultTimeoutCycles))
-      issue_pv<D, QUANT>(tmem + 128, tmem, smem_u32(smem), 0u);
+    if (mbar_wait(&bars[0], 0, &abort_s, kDefaultTimeoutCycles)) {
+      if constexpr (QUANT)
+        issue_pv_quant<D>(tmem + 128, smem_u32(p_tile), smem_u32(smem), 0u);
+      else
+        issue_pv_bf16<D>(tmem + 128, tmem, smem_u32(smem), 0u);
+    }
     mma_commit(&bars[1]);
   }
   __syncthreads();
@@ -569,7 +721,13 @@ cudaError_t launch_attn_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           int BH, cudaStream_t stream) {
   using C = Cfg<D, QUANT>;
   auto kern = attn_kernel<D, QUANT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  // the setmaxnreg split must fit in the registers the block is launched with,
+  // or the increase would wait forever
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * C::REGS_LOW + 256 * C::REGS_HIGH) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((prm.nT + 1) / 2, BH);
   kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
@@ -642,7 +800,7 @@ cudaError_t launch_dbg_pv_tile(const void* p, const void* vt, int d, int mode, f
     okm = encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vt, d, 128, (uint64_t)d * 2, 64, 128,
                          CU_TENSOR_MAP_SWIZZLE_128B);
   if (!okm) return cudaErrorInvalidValue;
-  const int smem = 128 * d * (quant ? 1 : 2) + 64 + 1024;
+  const int smem = 128 * d * (quant ? 1 : 2) + (quant ? 128 * 128 : 0) + 64 + 1024;
   const uint8_t* pp = static_cast<const uint8_t*>(p);
 #define SAGE_DBG_PV(DD, QQ)                                                                         \
   do {                                                                                              \
