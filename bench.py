@@ -38,9 +38,14 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "wan14b_720p"
-# Attention-kernel DRAM bytes per launch from an ncu capture, per workload;
-# None until a capture of the current kernel exists.
-NCU_TRAFFIC_BYTES = {}
+# Attention-kernel DRAM bytes (read + write) per full launch, from the ncu
+# captures summarised in profiles/attn_{i8f8,bf16}_wan14b_720p.md: a 4-head
+# capture of the same kernel, scaled by heads (each head's operands are read
+# from DRAM once).  Keyed by (workload, H, mode); absent keys report null.
+NCU_TRAFFIC_BYTES = {
+    ("wan14b_720p", 40, "int8_fp8"): 1.653e9,
+    ("wan14b_720p", 40, "bf16"): 3.002e9,
+}
 
 
 def parse():
@@ -52,7 +57,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--heads", type=int, default=0, help="override H (small profiling captures)")
     ap.add_argument("--mode", default="int8_fp8", choices=["int8_fp8", "bf16"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=3, help="end-to-end steps (at least 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4096)
     return ap.parse_args()
@@ -64,6 +69,22 @@ def workload(args):
         from dataclasses import replace
         w = replace(w, H=args.heads)
     return w
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank value over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Each rank attends over its own batch element: same shape, seed offset by rank."""
+    return w.with_seed(w.seed + rank)
 
 
 def load_peaks():
@@ -183,8 +204,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = workload(args)
     mode = sage.MODE_INT8_FP8 if args.mode == "int8_fp8" else sage.MODE_BF16
-    # every rank draws its own batch element: seed offset by rank
-    wr = w.with_seed(w.seed + rank)
+    wr = rank_workload(w, rank)
     q_h, k_h, v_h = synth.qkv_torch(wr, pin=True)
     q, k, v = (t.to(dev, non_blocking=True) for t in (q_h, k_h, v_h))
     o = torch.empty_like(q)
@@ -263,11 +283,7 @@ def run_ours(args, rank, world, local_rank):
     if st != sage.OK:
         raise sage.SageError(st, "timed region")
 
-    # max over ranks
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     # ---- end to end: pinned host inputs -> device -> public call -> host output ----
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -293,11 +309,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -345,6 +357,7 @@ def run_ours(args, rank, world, local_rank):
 
 def main():
     args = parse()
+    args.e2e_steps = max(1, args.e2e_steps)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
