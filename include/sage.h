@@ -21,7 +21,7 @@
  *    fixed scratch array of sage_quantize_qk_noalloc (see there).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Calls are asynchronous on that stream; no call synchronises except
- *    sage_status().
+ *    sage_status() and sage_attn_fwd_host().
  *  - Every function returns SAGE_OK (0) or a negative SAGE_E* code; none
  *    aborts or throws.  Argument errors are detected on the host before any
  *    launch.  Device-side failures (a bounded wait that ran out) are recorded
@@ -146,6 +146,26 @@ int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* 
  */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                   int mode, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The same call from host memory, pipelined: the B*H heads are processed in
+ * chunks of `chunk_heads` (0: B*H/8 rounded up); the host-to-device copy of
+ * chunk i+1 and the device-to-host copy of chunk i-1 overlap the attention of
+ * chunk i.  Heads are independent (every statistic of the scheme is per head),
+ * so the result is bit-for-bit that of sage_attn_fwd on the whole tensor.
+ * q_host, k_host, v_host, o_host: HOST bf16 [B,H,N,d]; pinned (page-locked)
+ *   memory is needed for the copies to overlap.
+ * q_dev, k_dev, v_dev, o_dev: device staging buffers bf16 [B,H,N,d] (caller-owned).
+ * workspace: at least sage_workspace_bytes(1, chunk_heads, N, d, mode) bytes,
+ *   reused by every chunk.
+ * Runs after earlier work on `stream` and returns when the output is in
+ * o_host (it synchronises); it creates and destroys two copy streams and
+ * three events, and allocates no device memory.  Returns the status of the
+ * call including device-side status (SAGE_ETIMEOUT).
+ */
+int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H,
+                       int N, int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                       void* workspace, size_t workspace_bytes, int chunk_heads, void* stream);
 
 /*
  * Per-layer mode table for selective quantization ("keeping video quality":

@@ -10,7 +10,7 @@ EXPECTED = {
     "sage_workspace_bytes", "sage_prepass_scratch_bytes", "sage_quantize_qk", "sage_attn_quantized",
     "sage_attn_fwd", "attn_layer_schedule", "sage_status", "sage_strerror", "sage_device_check",
     "sage_dbg_qk_tiles", "sage_dbg_pv_tile", "sage_dbg_qk_bf16_tile", "sage_dbg_attn_forced_timeout",
-    "sage_quantize_qk_noalloc",
+    "sage_quantize_qk_noalloc", "sage_attn_fwd_host",
 }
 
 

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -190,6 +191,75 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   if (e != cudaSuccess) return launch_status(e);
   return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
                                         kDefaultTimeoutCycles, 0, st));
+}
+
+int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H, int N,
+                       int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev, void* workspace,
+                       size_t workspace_bytes, int chunk_heads, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc != SAGE_OK) return rc;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8) return SAGE_EINVAL;
+  const void* ptrs[] = {q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  const int BH = B * H;
+  if (chunk_heads <= 0) chunk_heads = (BH + 7) / 8;
+  if (chunk_heads > BH) chunk_heads = BH;
+  const int n_chunks = (BH + chunk_heads - 1) / chunk_heads;
+  if (workspace_bytes < sage_workspace_bytes(1, chunk_heads, N, d, mode)) return SAGE_EWORKSPACE;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess) return SAGE_ELAUNCH;
+  if (cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaStreamDestroy(s_in);
+    return SAGE_ELAUNCH;
+  }
+  // inputs of chunk i land (s_in) -> its attention runs (stream) -> its output leaves (s_out)
+  cudaEvent_t ev_start, ev_in, ev_done;
+  cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
+  cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+  // copies may not start before earlier work on the caller's stream
+  cudaEventRecord(ev_start, st);
+  cudaStreamWaitEvent(s_in, ev_start, 0);
+  const size_t head_bytes = (size_t)N * d * 2;
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(o_host);
+  char* qd = static_cast<char*>(q_dev);
+  char* kd = static_cast<char*>(k_dev);
+  char* vd = static_cast<char*>(v_dev);
+  char* od = static_cast<char*>(o_dev);
+  rc = SAGE_OK;
+  for (int i = 0; i < n_chunks && rc == SAGE_OK; ++i) {
+    const int h0 = i * chunk_heads, hc = std::min(chunk_heads, BH - h0);
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hc * head_bytes;
+    if (cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(vd + off, vh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(st, ev_in, 0) != cudaSuccess) {
+      rc = SAGE_ELAUNCH;
+      break;
+    }
+    rc = sage_attn_fwd(qd + off, kd + off, vd + off, od + off, 1, hc, N, d, mode, workspace, workspace_bytes, stream);
+    if (rc != SAGE_OK) break;
+    if (cudaEventRecord(ev_done, st) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+      rc = SAGE_ELAUNCH;
+  }
+  // the caller's stream resumes after the last output copy
+  cudaEventRecord(ev_done, s_out);
+  cudaStreamWaitEvent(st, ev_done, 0);
+  if (cudaStreamSynchronize(s_out) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) rc = SAGE_ELAUNCH;
+  cudaEventDestroy(ev_start);
+  cudaEventDestroy(ev_in);
+  cudaEventDestroy(ev_done);
+  cudaStreamDestroy(s_in);
+  cudaStreamDestroy(s_out);
+  if (rc != SAGE_OK) return rc;
+  return sage_status(workspace, stream);
 }
 
 int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_fp, int8_t* modes_out) {

@@ -50,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "sage_dbg_qk_bf16_tile": (i32, [vp, vp, i32, vp, vp]),
         "sage_dbg_attn_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
         "sage_quantize_qk_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "sage_attn_fwd_host": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, i32, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -177,6 +178,29 @@ def attn_fwd(q, k, v, mode: int, o=None, workspace=None, stream=None):
     _check(LIB.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(mode), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)), "sage_attn_fwd")
     return o
+
+
+def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, chunk_heads: int = 0, stream=None):
+    """sage_attn_fwd_host: host bf16 [B,H,N,d] tensors (pinned for overlap) in, o_h filled on return.
+
+    staging: optional tuple of four device bf16 tensors shaped like q_h; workspace: optional
+    device buffer of sage_workspace_bytes(1, chunk, N, d, mode) bytes.
+    """
+    import torch
+    B, H, N, d = _bhnd(q_h, "q_h")
+    BH = B * H
+    chunk = chunk_heads if chunk_heads > 0 else (BH + 7) // 8
+    chunk = min(chunk, BH)
+    if staging is None:
+        staging = tuple(torch.empty(q_h.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    if workspace is None:
+        workspace = alloc_workspace(1, chunk, N, d, mode)
+    qd, kd, vd, od = staging
+    _check(LIB.sage_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), B, H, N, d, int(mode), _ptr(qd),
+                                  _ptr(kd), _ptr(vd), _ptr(od), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), int(chunk), _stream(stream)),
+           "sage_attn_fwd_host")
+    return o_h
 
 
 def status(workspace, stream=None) -> int:
