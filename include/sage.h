@@ -177,6 +177,32 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
 int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_fp, int8_t* modes_out);
 
 /*
+ * Per-layer error calibration for attn_layer_schedule ("keeping video
+ * quality": the quantized attention error of each layer is measured over the
+ * denoising iterations, and the layers whose error stays large keep the
+ * original precision).
+ *
+ * sage_attn_error_stats: a, b device bf16 [B,H,N,d] (16-byte aligned, d a
+ * multiple of 8); stats device fp64 [B*H][4] = per head
+ * {sum (a-b)^2, sum b^2, sum a*b, sum a^2} (e.g. a = INT8/FP8 output,
+ * b = BF16 output: relative L2 error = sqrt(s0/s1), cosine = s2/sqrt(s1*s3)).
+ * Deterministic (fixed summation order).  scratch: device buffer of
+ * sage_error_scratch_bytes(B, H) bytes.  Asynchronous on `stream`.
+ *
+ * sage_select_full_precision_layers: host layer_err [num_layers][num_iters]
+ * (any per-layer, per-iteration error, e.g. the relative L2 error above);
+ * writes, in ascending order, the layers whose mean error over the iterations
+ * exceeds `threshold` to host layers_out[num_layers] and their count to
+ * *n_out; the result feeds attn_layer_schedule.  SAGE_EINVAL on a non-finite
+ * error or bad sizes.
+ */
+size_t sage_error_scratch_bytes(int B, int H);
+int sage_attn_error_stats(const void* a, const void* b, int B, int H, int N, int d, double* stats,
+                          void* scratch, size_t scratch_bytes, void* stream);
+int sage_select_full_precision_layers(const double* layer_err, int num_layers, int num_iters,
+                                      double threshold, int* layers_out, int* n_out);
+
+/*
  * Reads and clears the device status word at the start of `workspace`
  * (synchronises `stream`).  Returns SAGE_OK, SAGE_ETIMEOUT if a bounded
  * device-side wait ran out since the last call, or SAGE_ELAUNCH if the stream

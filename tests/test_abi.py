@@ -10,7 +10,8 @@ EXPECTED = {
     "sage_workspace_bytes", "sage_prepass_scratch_bytes", "sage_quantize_qk", "sage_attn_quantized",
     "sage_attn_fwd", "attn_layer_schedule", "sage_status", "sage_strerror", "sage_device_check",
     "sage_dbg_qk_tiles", "sage_dbg_pv_tile", "sage_dbg_qk_bf16_tile", "sage_dbg_attn_forced_timeout",
-    "sage_quantize_qk_noalloc", "sage_attn_fwd_host",
+    "sage_quantize_qk_noalloc", "sage_attn_fwd_host", "sage_error_scratch_bytes", "sage_attn_error_stats",
+    "sage_select_full_precision_layers",
 }
 
 
@@ -66,3 +67,13 @@ def test_layer_schedule_host():
 def test_strerror_covers_codes():
     for c in (0, -1, -2, -3, -4, -5):
         assert sage.strerror(c) and sage.strerror(c) != "unknown status"
+
+
+def test_select_full_precision_layers_host():
+    err = [[0.01, 0.02], [0.30, 0.25], [0.05, 0.40], [0.2, 0.1]]
+    # means 0.015, 0.275, 0.225, 0.15
+    assert sage.select_full_precision_layers(err, 0.2) == [1, 2]
+    assert sage.select_full_precision_layers(err, 0.0) == [0, 1, 2, 3]
+    assert sage.select_full_precision_layers(err, 1.0) == []
+    with pytest.raises(sage.SageError):
+        sage.select_full_precision_layers([[float("nan")]], 0.1)

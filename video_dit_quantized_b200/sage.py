@@ -51,6 +51,9 @@ def _load() -> ctypes.CDLL:
         "sage_dbg_attn_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
         "sage_quantize_qk_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "sage_attn_fwd_host": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, i32, vp]),
+        "sage_error_scratch_bytes": (sz, [i32, i32]),
+        "sage_attn_error_stats": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "sage_select_full_precision_layers": (i32, [vp, i32, i32, ctypes.c_double, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -201,6 +204,50 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, c
                                   workspace.numel() * workspace.element_size(), int(chunk), _stream(stream)),
            "sage_attn_fwd_host")
     return o_h
+
+
+def error_stats(a, b, stream=None):
+    """Per-head fp64 [B*H, 4] = {sum (a-b)^2, sum b^2, sum a*b, sum a^2} of two bf16 [B,H,N,d] tensors (device)."""
+    import torch
+    B, H, N, d = _bhnd(a, "a")
+    stats = torch.empty((B * H, 4), dtype=torch.float64, device=a.device)
+    scratch = torch.empty(max(int(LIB.sage_error_scratch_bytes(B, H)), 16), dtype=torch.uint8, device=a.device)
+    _check(LIB.sage_attn_error_stats(_ptr(a), _ptr(b), B, H, N, d, _ptr(stats), _ptr(scratch), scratch.numel(),
+                                     _stream(stream)), "sage_attn_error_stats")
+    return stats
+
+
+def layer_errors(layers, stream=None):
+    """Relative L2 error of the INT8/FP8 output against the BF16 output, per layer and iteration.
+
+    layers: [num_layers][num_iters] of (q, k, v) device bf16 [B,H,N,d] tensors.
+    Returns a nested list [num_layers][num_iters] of sqrt(sum (a-b)^2 / sum b^2) over all heads.
+    """
+    out = []
+    for per_layer in layers:
+        row = []
+        for (q, k, v) in per_layer:
+            oq = attn_fwd(q, k, v, MODE_INT8_FP8, stream=stream)
+            ob = attn_fwd(q, k, v, MODE_BF16, stream=stream)
+            st = error_stats(oq, ob, stream=stream).sum(dim=0).cpu()
+            row.append(float((st[0] / st[1]).sqrt()))
+        out.append(row)
+    return out
+
+
+def select_full_precision_layers(layer_err, threshold: float) -> list[int]:
+    """Layers whose mean error over iterations exceeds threshold; layer_err is [layers][iterations]."""
+    import numpy as np
+    err = np.ascontiguousarray(np.asarray(layer_err, dtype=np.float64))
+    if err.ndim != 2:
+        raise ValueError("layer_err must be [layers][iterations]")
+    L, I = err.shape
+    out = (ctypes.c_int * max(L, 1))()
+    n = ctypes.c_int(0)
+    _check(LIB.sage_select_full_precision_layers(err.ctypes.data_as(ctypes.c_void_p), L, I, float(threshold),
+                                                 ctypes.cast(out, ctypes.c_void_p), ctypes.byref(n)),
+           "sage_select_full_precision_layers")
+    return [int(out[i]) for i in range(n.value)]
 
 
 def status(workspace, stream=None) -> int:
