@@ -35,6 +35,7 @@ EMUL_P_FP32 = 1
 EMUL_V_EXACT = 2
 EMUL_QK_EXACT = 4
 EMUL_ONE_TILE = 8
+EMUL_Q_PER_TOKEN = 16
 
 
 def build(force: bool = False) -> str:
@@ -67,6 +68,7 @@ def _load():
             lib.orc_k_mean.argtypes = [u16, i32, i32, i32, i32, f32]
             lib.orc_quant_int8_blocks.argtypes = [u16, f32, i32, i32, i32, i32, i8, f32]
             lib.orc_quant_v_fp8.argtypes = [u16, i32, i32, i32, i32, u8, f32]
+            lib.orc_quant_int8_rows.argtypes = [u16, f32, i32, i32, i32, i32, i32, i8, f32]
             lib.orc_qk_tile.argtypes = [i8, i8, i32, i32, i64, i32, i32, s32]
             lib.orc_attn_exact.argtypes = [u16, u16, u16, i32, i32, i32, i32, P(i32), i32, f64]
             lib.orc_attn_emul.argtypes = [i8, f32, i8, f32, u8, f32, i32, i32, i32, i32, P(i32), i32, i32,
@@ -122,6 +124,19 @@ def quant_int8_blocks(x: np.ndarray, mean: np.ndarray | None = None):
     return codes, scale
 
 
+def quant_int8_rows(x: np.ndarray, rows: int, mean: np.ndarray | None = None):
+    """INT8 codes [B,H,N,d] and fp32 scales [B,H,ceil(N/rows)] with a block of `rows` tokens (1: per token)."""
+    x = _c(x, np.uint16)
+    B, H, N, d = x.shape
+    nb = (N + rows - 1) // rows
+    codes = np.empty((B, H, N, d), dtype=np.int8)
+    scale = np.empty((B, H, nb), dtype=np.float32)
+    m = None if mean is None else _c(mean, np.float32)
+    _load().orc_quant_int8_rows(_p(x, ctypes.c_uint16), _p(m, ctypes.c_float), B, H, N, d, int(rows),
+                                _p(codes, ctypes.c_int8), _p(scale, ctypes.c_float))
+    return codes, scale
+
+
 def quant_v_fp8(v: np.ndarray):
     """a4: e4m3 codes [B,H,N,d] (natural layout) and fp32 per-channel scales [B,H,d]."""
     v = _c(v, np.uint16)
@@ -133,10 +148,14 @@ def quant_v_fp8(v: np.ndarray):
     return codes, scale
 
 
-def prepass(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
-    """a1..a4 in order; returns every intermediate the path exposes."""
+def prepass(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_per_token: bool = False) -> dict:
+    """a1..a4 in order; returns every intermediate the path exposes.
+
+    q_per_token: one Q scale per token instead of per 128-token block (the
+    finer granularity; pair it with attn_emul(..., flags=EMUL_Q_PER_TOKEN)).
+    """
     mean = k_mean(k)
-    q8, qs = quant_int8_blocks(q)
+    q8, qs = quant_int8_rows(q, 1) if q_per_token else quant_int8_blocks(q)
     k8, ks = quant_int8_blocks(k, mean)
     v8, vs = quant_v_fp8(v)
     return dict(k_mean=mean, q_i8=q8, q_scale=qs, k_i8=k8, k_scale=ks, v_f8=v8, v_scale=vs)

@@ -167,6 +167,50 @@ void orc_quant_int8_blocks(const uint16_t* x, const float* mean, int B, int H, i
     }
 }
 
+/*
+ * The same quantization with a block of `rows` consecutive tokens (rows = 1:
+ * one scale per token, the finer Q granularity).  codes: int8 [B,H,N,d];
+ * scale: fp32 [B,H,ceil(N/rows)].  Same formula and zero guard as above.
+ */
+void orc_quant_int8_rows(const uint16_t* x, const float* mean, int B, int H, int N, int d, int rows,
+                         int8_t* codes, float* scale) {
+    long BH = (long)B * H;
+    int nb = (N + rows - 1) / rows;
+#pragma omp parallel for schedule(static)
+    for (long blk = 0; blk < BH * nb; ++blk) {
+        long bh = blk / nb;
+        int b0 = (int)(blk % nb) * rows;
+        int b1 = b0 + rows < N ? b0 + rows : N;
+        const uint16_t* xh = x + bh * (long)N * d;
+        const float* mh = mean ? mean + bh * d : NULL;
+        float amax = 0.0f;
+        for (int n = b0; n < b1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float v = bf16f(xh[(long)n * d + c]);
+                if (mh) v = v - mh[c];
+                float a = fabsf(v);
+                if (a > amax) amax = a;
+            }
+        int8_t* ch = codes + bh * (long)N * d;
+        if (amax == 0.0f) {
+            scale[blk] = 0.0f;
+            for (int n = b0; n < b1; ++n) memset(ch + (long)n * d, 0, (size_t)d);
+            continue;
+        }
+        float inv = 127.0f / amax;
+        scale[blk] = amax / 127.0f;
+        for (int n = b0; n < b1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float v = bf16f(xh[(long)n * d + c]);
+                if (mh) v = v - mh[c];
+                double r = rne((double)(v * inv));
+                if (r > 127.0) r = 127.0;
+                if (r < -127.0) r = -127.0;
+                ch[(long)n * d + c] = (int8_t)r;
+            }
+    }
+}
+
 /* ---------------- a4: per-channel FP8 V ---------------- */
 
 /* v: bf16 [B,H,N,d] -> codes e4m3 [B,H,N,d] (natural layout), scale fp32 [B,H,d] */
@@ -267,7 +311,9 @@ void orc_attn_exact(const uint16_t* q, const uint16_t* k, const uint16_t* v, int
  * flags: bit 0 keep P in fp32 (skip a7's e4m3 rounding, scale stays 448),
  *        bit 1 use dequantized-exact V (v8 * v_scale replaced by bf16 V; needs v_bf16),
  *        bit 2 use the bf16 Q/K instead of the INT8 codes (needs q_bf16/k_bf16),
- *        bit 3 one key tile spanning all N (no tiling of the online softmax).
+ *        bit 3 one key tile spanning all N (no tiling of the online softmax),
+ *        bit 4 q_scale holds one scale per query token ([B*H, N]) instead of
+ *              one per 128-token block (the finer Q granularity).
  * The bits exist only to pin the emulation against O1 as quantization is
  * switched off step by step.
  *
@@ -319,7 +365,8 @@ void orc_attn_emul(const int8_t* q8, const float* q_scale, const int8_t* k8, con
                     } else {
                         int32_t S = 0;
                         for (int c = 0; c < d; ++c) S += (int32_t)qh[(long)i * d + c] * (int32_t)kh[(long)j * d + c];
-                        float sc = q_scale[bh * nT + qb] * k_scale[bh * nT + j / ORC_TILE];
+                        float qsc = (flags & 16) ? q_scale[bh * (long)N + i] : q_scale[bh * nT + qb];
+                        float sc = qsc * k_scale[bh * nT + j / ORC_TILE];
                         sc = sc * c_scale;
                         sj = (float)S * sc;
                     }

@@ -181,3 +181,29 @@ def test_layer_schedule():
         oracle.layer_schedule(4, [4])
     with pytest.raises(ValueError):
         oracle.layer_schedule(4, [-1])
+
+
+def test_per_token_q_scale_emulation():
+    # every row of a block shares its absmax -> per-token scales equal the block scale,
+    # so the per-token emulation must equal the per-block one exactly
+    w = synth.Workload("t", 1, 2, 256, 64, seed=17)
+    q, k, v = synth.qkv_numpy(w)
+    Q = synth.bf16_bits_to_f32(q).copy()
+    Q = np.clip(Q, -3.0, 3.0)
+    Q[..., 0] = 4.0
+    q = bf16(Q)
+    pre_b = oracle.prepass(q, k, v)
+    pre_t = oracle.prepass(q, k, v, q_per_token=True)
+    assert np.array_equal(pre_b["q_i8"], pre_t["q_i8"])
+    assert np.all(pre_t["q_scale"] == pre_b["q_scale"][0, 0, 0])
+    rows = [0, 5, 130, 255]
+    ob, _ = oracle.attn_emul(pre_b, rows)
+    ot, _ = oracle.attn_emul(pre_t, rows, flags=oracle.EMUL_Q_PER_TOKEN)
+    np.testing.assert_array_equal(ob, ot)
+    # on ordinary inputs the per-token scheme stays close to exact attention
+    w = synth.Workload("t", 1, 2, 700, 128, seed=18, outlier_frac=0.01)
+    q, k, v = synth.qkv_numpy(w)
+    rows = synth.sample_rows(4, w.N, 64)
+    o1 = oracle.attn_exact(q, k, v, rows)
+    ot, _ = oracle.attn_emul(oracle.prepass(q, k, v, q_per_token=True), rows, flags=oracle.EMUL_Q_PER_TOKEN)
+    assert cos(ot, o1) >= 0.995

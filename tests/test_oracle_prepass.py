@@ -159,3 +159,27 @@ def test_v_fp8_per_channel():
                 best = np.flatnonzero(dist == dist.min())
                 want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
                 assert code & 0x7F == want
+
+
+def test_rows_quantizer_generalises_the_block_one():
+    (q, k, v), w = _tiny_tensor(15, 2, 2, 300, 64)
+    a = oracle.quant_int8_blocks(q)
+    b = oracle.quant_int8_rows(q, 128)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+    mean = oracle.k_mean(k)
+    a = oracle.quant_int8_blocks(k, mean)
+    b = oracle.quant_int8_rows(k, 128, mean)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+
+
+def test_per_token_q_int8():
+    (q, k, v), w = _tiny_tensor(16, 1, 2, 70, 32)
+    q = q.copy()
+    q[0, 1, 5] = 0                                       # an all-zero token
+    codes, scale = oracle.quant_int8_rows(q, 1)
+    assert scale.shape == (1, 2, 70)
+    qf = synth.bf16_bits_to_f32(q)
+    for h in range(2):
+        for n in range(70):
+            _check_int8_block_properties(qf[0, h, n:n + 1], codes[0, h, n:n + 1], float(scale[0, h, n]))
+    assert scale[0, 1, 5] == 0.0 and not codes[0, 1, 5].any()
