@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--heads", type=int, default=0, help="override H (small profiling captures)")
-    ap.add_argument("--mode", default="int8_fp8", choices=["int8_fp8", "bf16"])
+    ap.add_argument("--mode", default="int8_fp8", choices=["int8_fp8", "bf16", "int8_fp8_qtoken"])
     ap.add_argument("--e2e-steps", type=int, default=3, help="end-to-end steps (at least 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4096)
@@ -203,7 +203,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = workload(args)
-    mode = sage.MODE_INT8_FP8 if args.mode == "int8_fp8" else sage.MODE_BF16
+    mode = {"int8_fp8": sage.MODE_INT8_FP8, "bf16": sage.MODE_BF16, "int8_fp8_qtoken": sage.MODE_INT8_FP8_QTOKEN}[args.mode]
+    quant = mode != sage.MODE_BF16
+    qgran = 1 if mode == sage.MODE_INT8_FP8_QTOKEN else 128
     wr = rank_workload(w, rank)
     q_h, k_h, v_h = synth.qkv_torch(wr, pin=True)
     q, k, v = (t.to(dev, non_blocking=True) for t in (q_h, k_h, v_h))
@@ -212,10 +214,10 @@ def run_ours(args, rank, world, local_rank):
     ws = sage.alloc_workspace(w.B, w.H, w.N, w.d, mode, dev)
     nT = (w.N + 127) // 128
     pre = None
-    if mode == sage.MODE_INT8_FP8:
+    if quant:
         pre = dict(
             q_i8=torch.empty((w.B, w.H, nT * 128, w.d), dtype=torch.int8, device=dev),
-            q_scale=torch.empty((w.B, w.H, nT), dtype=torch.float32, device=dev),
+            q_scale=torch.empty((w.B, w.H, nT * 128 if qgran == 1 else nT), dtype=torch.float32, device=dev),
             k_i8=torch.empty((w.B, w.H, nT * 128, w.d), dtype=torch.int8, device=dev),
             k_scale=torch.empty((w.B, w.H, nT), dtype=torch.float32, device=dev),
             k_mean=torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev),
@@ -232,18 +234,19 @@ def run_ours(args, rank, world, local_rank):
         """One pass of the path; ev = (start, after_prepass, end) events or None."""
         if ev:
             ev[0].record(stream)
-        if mode == sage.MODE_INT8_FP8:
-            rc = sage.LIB.sage_quantize_qk(P(q), P(k), P(v), w.B, w.H, w.N, w.d, P(pre["q_i8"]), P(pre["q_scale"]),
-                                           P(pre["k_i8"]), P(pre["k_scale"]), P(pre["k_mean"]), P(pre["v_f8t"]),
-                                           P(pre["v_scale"]), P(scratch), scratch.numel(), sp)
+        if quant:
+            rc = sage.LIB.sage_quantize_qk_ex(P(q), P(k), P(v), w.B, w.H, w.N, w.d, qgran, P(pre["q_i8"]),
+                                              P(pre["q_scale"]), P(pre["k_i8"]), P(pre["k_scale"]), P(pre["k_mean"]),
+                                              P(pre["v_f8t"]), P(pre["v_scale"]), P(scratch), scratch.numel(), sp)
             if rc:
-                raise sage.SageError(rc, "sage_quantize_qk")
+                raise sage.SageError(rc, "sage_quantize_qk_ex")
             if ev:
                 ev[1].record(stream)
-            rc = sage.LIB.sage_attn_quantized(P(pre["q_i8"]), P(pre["q_scale"]), P(pre["k_i8"]), P(pre["k_scale"]),
-                                              P(pre["v_f8t"]), P(pre["v_scale"]), P(o), w.B, w.H, w.N, w.d, P(ws), sp)
+            rc = sage.LIB.sage_attn_quantized_ex(P(pre["q_i8"]), P(pre["q_scale"]), P(pre["k_i8"]),
+                                                 P(pre["k_scale"]), P(pre["v_f8t"]), P(pre["v_scale"]), P(o), w.B, w.H,
+                                                 w.N, w.d, qgran, P(ws), sp)
             if rc:
-                raise sage.SageError(rc, "sage_attn_quantized")
+                raise sage.SageError(rc, "sage_attn_quantized_ex")
         else:
             if ev:
                 ev[1].record(stream)
@@ -326,7 +329,7 @@ def run_ours(args, rank, world, local_rank):
     # dense contraction peak for the kernel's own dtype: INT8/FP8 = 2x the measured
     # bf16 figure (nominal 4.5 vs 2.25 PFLOP/s); the sustained figure, since the
     # kernel runs back to back for seconds under the power cap.
-    ratio = 2.0 if mode == sage.MODE_INT8_FP8 else 1.0
+    ratio = 2.0 if quant else 1.0
     peak = ratio * float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     attn_avg = statistics.mean(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
@@ -336,7 +339,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": "attention TFLOPS per call (4*B*H*N^2*d)",
         "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8/fp8e4m3 (fp32 accumulate)" if mode == sage.MODE_INT8_FP8 else "bf16 (fp32 accumulate)",
+        "dtype": "int8/fp8e4m3 (fp32 accumulate)" if quant else "bf16 (fp32 accumulate)",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
                    "global_batch": world * w.B, "parallelism": f"independent calls x{world}",
@@ -350,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * (4 if mode == sage.MODE_INT8_FP8 else 1),
+        "gpu_launches": args.steps * (4 if quant else 1),
         "e2e_api": "sage_attn_fwd_host (pinned host Q/K/V in, O out, pipelined over 8 head chunks)",
         "clocks": clocks,
     }

@@ -40,6 +40,7 @@ extern "C" {
 /* attention modes (one per layer, see attn_layer_schedule) */
 #define SAGE_MODE_BF16 0      /* exact softmax attention, BF16 tensor-core MMAs */
 #define SAGE_MODE_INT8_FP8 1  /* smoothed INT8 QK^T, FP8 e4m3 P.V             */
+#define SAGE_MODE_INT8_FP8_QTOKEN 2  /* the same with one Q scale per token  */
 
 /* status codes */
 #define SAGE_OK 0
@@ -87,6 +88,19 @@ size_t sage_workspace_bytes(int B, int H, int N, int d, int mode);
  * with nQ = nK = ceil(N/128).
  */
 size_t sage_prepass_scratch_bytes(int B, int H, int N, int d);
+/*
+ * The prepass with a choice of Q granularity: q_granularity = 128 is
+ * sage_quantize_qk (one Q scale per 128-token block, q_scale [B,H,nQ]);
+ * q_granularity = 1 gives one Q scale per token, amax over the token's d
+ * channels / 127 with the same rounding and zero guard, q_scale [B,H,nQ*128]
+ * (rows >= N get scale 0).  This finer granularity costs nothing in the
+ * attention kernel, where each thread owns one query row.  Other values:
+ * SAGE_EINVAL.
+ */
+int sage_quantize_qk_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        int q_granularity, int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                        float* k_mean, uint8_t* v_f8t, float* v_scale, void* scratch, size_t scratch_bytes,
+                        void* stream);
 int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                      int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
                      uint8_t* v_f8t, float* v_scale, void* scratch, size_t scratch_bytes,
@@ -132,12 +146,18 @@ int sage_quantize_qk_noalloc(const void* q, const void* k, const void* v, int B,
 int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
                         const float* k_scale, const uint8_t* v_f8t, const float* v_scale,
                         void* o, int B, int H, int N, int d, void* status, void* stream);
+/* The same with q_scale in the granularity sage_quantize_qk_ex wrote (128 or 1). */
+int sage_attn_quantized_ex(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                           const float* k_scale, const uint8_t* v_f8t, const float* v_scale, void* o, int B,
+                           int H, int N, int d, int q_granularity, void* status, void* stream);
 
 /*
  * Full-sequence self-attention O = softmax(Q K^T / sqrt(d)) V, non-causal,
  * q, k, v, o bf16 [B,H,N,d].
  * mode SAGE_MODE_INT8_FP8: sage_quantize_qk into the workspace, then
  *   sage_attn_quantized.
+ * mode SAGE_MODE_INT8_FP8_QTOKEN: the same with one Q scale per token
+ *   (sage_quantize_qk_ex with q_granularity 1).
  * mode SAGE_MODE_BF16: S = Q K^T with BF16 tensor-core MMAs (fp32
  *   accumulate), online softmax in fp32, P rounded to bf16, O += P V
  *   (fp32), O / l rounded to bf16.  Uses only the status word of the workspace.

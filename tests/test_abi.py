@@ -11,7 +11,7 @@ EXPECTED = {
     "sage_attn_fwd", "attn_layer_schedule", "sage_status", "sage_strerror", "sage_device_check",
     "sage_dbg_qk_tiles", "sage_dbg_pv_tile", "sage_dbg_qk_bf16_tile", "sage_dbg_attn_forced_timeout",
     "sage_quantize_qk_noalloc", "sage_attn_fwd_host", "sage_error_scratch_bytes", "sage_attn_error_stats",
-    "sage_select_full_precision_layers",
+    "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
 }
 
 

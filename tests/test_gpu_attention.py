@@ -143,3 +143,40 @@ def test_layer_stack_schedule(cuda_dev):
                 _, o2, o1 = emul_and_exact(qh, kh, vh, rows)
                 check_quant(got, o2, o1, synth.bf16_bits_to_f32(vh), f"layer {layer}")
     assert sage.status(ws) == sage.OK
+
+
+def _emul_tok(q, k, v, rows):
+    pre = oracle.prepass(q, k, v, q_per_token=True)
+    o2, _ = oracle.attn_emul(pre, rows, flags=oracle.EMUL_Q_PER_TOKEN)
+    return o2, oracle.attn_exact(q, k, v, rows)
+
+
+@pytest.mark.parametrize("w", small_workloads(), ids=lambda w: w.name)
+def test_quantized_per_token_q_small_all_rows(w, cuda_dev):
+    import torch
+    from video_dit_quantized_b200 import sage
+    q, k, v = synth.qkv_numpy(w)
+    o2, o1 = _emul_tok(q, k, v, np.arange(w.N, dtype=np.int32))
+    qd, kd, vd = _dev(q, cuda_dev), _dev(k, cuda_dev), _dev(v, cuda_dev)
+    ws = sage.alloc_workspace(w.B, w.H, w.N, w.d, sage.MODE_INT8_FP8_QTOKEN)
+    o = sage.attn_fwd(qd, kd, vd, sage.MODE_INT8_FP8_QTOKEN, workspace=ws)
+    assert sage.status(ws) == sage.OK
+    check_quant(bf16_to_np(o), o2, o1, synth.bf16_bits_to_f32(v), w.name + " per-token Q")
+    pre = sage.quantize_qk(qd, kd, vd, q_per_token=True)
+    o_b = sage.attn_quantized(pre, w.N)
+    torch.cuda.synchronize()
+    assert torch.equal(o_b.view(torch.int16), o.view(torch.int16))
+
+
+def test_quantized_per_token_q_full_size_sampled(cuda_dev, big_inputs):
+    import torch
+    from video_dit_quantized_b200 import sage
+    name = "wan1.3b_480p"
+    w = synth.WORKLOADS[name]
+    q, k, v, qd, kd, vd = big_inputs(name)
+    hs = [0, w.H - 1]
+    rows = synth.sample_rows(w.seed + 98, w.N, 32)
+    o2, o1 = _emul_tok(heads(q, hs), heads(k, hs), heads(v, hs), rows)
+    o = sage.attn_fwd(qd, kd, vd, sage.MODE_INT8_FP8_QTOKEN)
+    got = bf16_to_np(o[:, hs][:, :, torch.from_numpy(rows).long().to(cuda_dev)])
+    check_quant(got, o2, o1, synth.bf16_bits_to_f32(heads(v, hs)), name + " per-token Q")

@@ -17,7 +17,7 @@ def test_host_pipeline_matches_device_call(w, chunk, cuda_dev):
     from video_dit_quantized_b200 import sage
     qh, kh, vh = synth.qkv_torch(w, pin=True)
     qd, kd, vd = (t.to(cuda_dev) for t in (qh, kh, vh))
-    for mode in (sage.MODE_INT8_FP8, sage.MODE_BF16):
+    for mode in (sage.MODE_INT8_FP8, sage.MODE_BF16, sage.MODE_INT8_FP8_QTOKEN):
         ref = sage.attn_fwd(qd, kd, vd, mode)
         oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
         sage.attn_fwd_host(qh, kh, vh, oh, mode, chunk_heads=chunk)

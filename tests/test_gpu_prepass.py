@@ -72,3 +72,22 @@ def test_prepass_bit_exact_full_size(name, cuda_dev, big_inputs):
     hs = sorted({0, w.H // 2, w.H - 1})
     pre_o = oracle.prepass(heads(q, hs), heads(k, hs), heads(v, hs))
     compare_prepass(pre_g, pre_o, w.N, hs)
+
+
+@pytest.mark.parametrize("w", small_workloads(), ids=lambda w: w.name)
+def test_prepass_per_token_q_bit_exact(w, cuda_dev):
+    """The finer Q granularity: one INT8 scale per token (amax of its d channels / 127)."""
+    import torch
+    from video_dit_quantized_b200 import sage
+    q, k, v = synth.qkv_numpy(w)
+    pre_o = oracle.prepass(q, k, v, q_per_token=True)
+    pre_g = sage.quantize_qk(_dev(q, cuda_dev), _dev(k, cuda_dev), _dev(v, cuda_dev), q_per_token=True)
+    torch.cuda.synchronize()
+    qs = pre_g["q_scale"].cpu().numpy()
+    np.testing.assert_array_equal(qs[:, :, :w.N].view(np.uint32), pre_o["q_scale"].view(np.uint32))
+    assert not qs[:, :, w.N:].any()
+    np.testing.assert_array_equal(pre_g["q_i8"].cpu().numpy()[:, :, :w.N], pre_o["q_i8"])
+    # K and V are the same as in the per-block prepass
+    ref = oracle.prepass(q, k, v)
+    for name in ("k_scale", "k_mean", "v_scale"):
+        np.testing.assert_array_equal(pre_g[name].cpu().numpy().view(np.uint32), ref[name].view(np.uint32))

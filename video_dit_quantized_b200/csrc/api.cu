@@ -38,7 +38,7 @@ struct Layout {
   size_t status, q_i8, k_i8, v_f8t, q_scale, k_scale, k_mean, v_scale, scratch, total;
 };
 
-Layout layout(int B, int H, int N, int d) {
+Layout layout(int B, int H, int N, int d, bool q_per_token = false) {
   const size_t BH = (size_t)B * H, nT = num_tiles(N), Npad = nT * kTile;
   Layout L;
   size_t off = 0;
@@ -51,7 +51,7 @@ Layout layout(int B, int H, int N, int d) {
   L.q_i8 = take(BH * Npad * d);
   L.k_i8 = take(BH * Npad * d);
   L.v_f8t = take(BH * d * Npad);
-  L.q_scale = take(BH * nT * 4);
+  L.q_scale = take(BH * (q_per_token ? Npad : nT) * 4);
   L.k_scale = take(BH * nT * 4);
   L.k_mean = take(BH * d * 4);
   L.v_scale = take(BH * d * 4);
@@ -124,6 +124,7 @@ size_t sage_workspace_bytes(int B, int H, int N, int d, int mode) {
   if (check_shape(B, H, N, d) != SAGE_OK) return 0;
   if (mode == SAGE_MODE_BF16) return 256;
   if (mode == SAGE_MODE_INT8_FP8) return layout(B, H, N, d).total;
+  if (mode == SAGE_MODE_INT8_FP8_QTOKEN) return layout(B, H, N, d, true).total;
   return 0;
 }
 
@@ -135,6 +136,14 @@ size_t sage_prepass_scratch_bytes(int B, int H, int N, int d) {
 int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, int N, int d, int8_t* q_i8,
                      float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t, float* v_scale,
                      void* scratch, size_t scratch_bytes, void* stream) {
+  return sage_quantize_qk_ex(q, k, v, B, H, N, d, SAGE_BLK_Q, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale,
+                             scratch, scratch_bytes, stream);
+}
+
+int sage_quantize_qk_ex(const void* q, const void* k, const void* v, int B, int H, int N, int d, int q_granularity,
+                        int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
+                        float* v_scale, void* scratch, size_t scratch_bytes, void* stream) {
+  if (q_granularity != SAGE_BLK_Q && q_granularity != 1) return SAGE_EINVAL;
   int rc = check_shape(B, H, N, d);
   if (rc != SAGE_OK) return rc;
   const void* ptrs[] = {q, k, v, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch};
@@ -144,12 +153,20 @@ int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, 
   if ((rc = check_device()) != SAGE_OK) return rc;
   const PrepassScratch s = prepass_scratch_carve(scratch, B * H, N, d);
   return launch_status(launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale,
-                                      s, static_cast<cudaStream_t>(stream)));
+                                      s, static_cast<cudaStream_t>(stream), q_granularity == 1));
 }
 
 int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
                         const uint8_t* v_f8t, const float* v_scale, void* o, int B, int H, int N, int d, void* status,
                         void* stream) {
+  return sage_attn_quantized_ex(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B, H, N, d, SAGE_BLK_Q, status,
+                                stream);
+}
+
+int sage_attn_quantized_ex(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                           const uint8_t* v_f8t, const float* v_scale, void* o, int B, int H, int N, int d,
+                           int q_granularity, void* status, void* stream) {
+  if (q_granularity != SAGE_BLK_Q && q_granularity != 1) return SAGE_EINVAL;
   int rc = check_shape(B, H, N, d);
   if (rc != SAGE_OK) return rc;
   const void* ptrs[] = {q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, status};
@@ -158,14 +175,14 @@ int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* 
   if ((rc = check_device()) != SAGE_OK) return rc;
   return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d,
                                         static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
-                                        static_cast<cudaStream_t>(stream)));
+                                        static_cast<cudaStream_t>(stream), q_granularity == 1));
 }
 
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int mode,
                   void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_shape(B, H, N, d);
   if (rc != SAGE_OK) return rc;
-  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8) return SAGE_EINVAL;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_INT8_FP8_QTOKEN) return SAGE_EINVAL;
   const void* ptrs[] = {q, k, v, o, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAGE_EINVAL;
@@ -177,7 +194,8 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   if (mode == SAGE_MODE_BF16)
     return launch_status(launch_attn_bf16(q, k, v, o, B * H, N, d, status, kDefaultTimeoutCycles, st));
-  const Layout L = layout(B, H, N, d);
+  const bool qtok = mode == SAGE_MODE_INT8_FP8_QTOKEN;
+  const Layout L = layout(B, H, N, d, qtok);
   auto q_i8 = reinterpret_cast<int8_t*>(ws + L.q_i8);
   auto k_i8 = reinterpret_cast<int8_t*>(ws + L.k_i8);
   auto v_f8t = reinterpret_cast<uint8_t*>(ws + L.v_f8t);
@@ -187,10 +205,10 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   auto v_scale = reinterpret_cast<float*>(ws + L.v_scale);
   const PrepassScratch s = prepass_scratch_carve(ws + L.scratch, B * H, N, d);
   cudaError_t e =
-      launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st);
+      launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st, qtok);
   if (e != cudaSuccess) return launch_status(e);
   return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
-                                        kDefaultTimeoutCycles, 0, st));
+                                        kDefaultTimeoutCycles, 0, st, qtok));
 }
 
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H, int N,
@@ -198,7 +216,7 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
                        size_t workspace_bytes, int chunk_heads, void* stream) {
   int rc = check_shape(B, H, N, d);
   if (rc != SAGE_OK) return rc;
-  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8) return SAGE_EINVAL;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_INT8_FP8_QTOKEN) return SAGE_EINVAL;
   const void* ptrs[] = {q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAGE_EINVAL;

@@ -148,6 +148,7 @@ struct Params {
   int N, nT, Npad;
   long long timeout;
   int dbg_flags;          // bit 0: MMA thread first waits on a barrier nobody arrives on
+  int q_per_token;        // QUANT: q_scale is [BH, Npad] (one scale per query token), else [BH, nT]
 };
 
 template <int D, bool QUANT>
@@ -344,7 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qt = qt0 + t;
     const float c = softmax_c(D);
     float qs = 1.0f;
-    if constexpr (QUANT) qs = qt < nT ? prm.q_scale[(size_t)bh * nT + qt] : 0.f;
+    if constexpr (QUANT) {
+      if (qt < nT)
+        qs = prm.q_per_token ? prm.q_scale[(size_t)bh * prm.Npad + qt * 128 + row] : prm.q_scale[(size_t)bh * nT + qt];
+      else
+        qs = 0.f;
+    }
     // QUANT: p is produced already multiplied by the P scale 448 (2^(s - m + log2 448)),
     // so l accumulates 448 * sum(p) and the epilogue divides by it directly.
     constexpr float kLog2PScale = QUANT ? 8.807354922057604f : 0.f;
@@ -738,7 +744,8 @@ cudaError_t launch_attn_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 
 cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
                              const uint8_t* v_f8t, const float* v_scale, void* o, int BH, int N, int d,
-                             uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream) {
+                             uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream,
+                             bool q_per_token) {
   const int nT = num_tiles(N), Npad = nT * kTile;
   alignas(64) CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -747,7 +754,8 @@ cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int
       !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, v_f8t, Npad, (uint64_t)BH * d, Npad, 128, d,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  Params prm{q_scale, k_scale, v_scale, static_cast<__nv_bfloat16*>(o), status, N, nT, Npad, timeout_cycles, dbg_flags};
+  Params prm{q_scale, k_scale, v_scale, static_cast<__nv_bfloat16*>(o), status, N, nT, Npad, timeout_cycles, dbg_flags,
+             q_per_token ? 1 : 0};
   if (d == 128) return launch_attn_d<128, true>(tq, tk, tv, prm, BH, stream);
   if (d == 64) return launch_attn_d<64, true>(tq, tk, tv, prm, BH, stream);
   return cudaErrorInvalidValue;
@@ -765,7 +773,7 @@ cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, void* 
       !encode_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, d, N, BH, s1, s2, 64, 128, 1,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  Params prm{nullptr, nullptr, nullptr, static_cast<__nv_bfloat16*>(o), status, N, nT, nT * kTile, timeout_cycles, 0};
+  Params prm{nullptr, nullptr, nullptr, static_cast<__nv_bfloat16*>(o), status, N, nT, nT * kTile, timeout_cycles, 0, 0};
   if (d == 128) return launch_attn_d<128, false>(tq, tk, tv, prm, BH, stream);
   if (d == 64) return launch_attn_d<64, false>(tq, tk, tv, prm, BH, stream);
   return cudaErrorInvalidValue;

@@ -28,14 +28,17 @@ struct PrepassScratch {
 size_t prepass_scratch_bytes(int BH, int N, int d);
 PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d);
 
+// q_per_token: q_scale is [BH, Npad] (one scale per token) instead of [BH, nT].
 cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
                            float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
-                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream);
+                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream,
+                           bool q_per_token = false);
 
 // Quantized attention (INT8 QK^T, FP8 PV).  status: device uint32 word.
 cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
                              const uint8_t* v_f8t, const float* v_scale, void* o, int BH, int N, int d,
-                             uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream);
+                             uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream,
+                             bool q_per_token = false);
 
 // BF16 attention.
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N, int d,

@@ -60,8 +60,9 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
-// grid (nK, BH)
-template <int D>
+// grid (nK, BH).  TOKQ: Q gets one scale per token (q_scale [BH, Npad]) instead
+// of one per 128-token block (q_scale [BH, nK]).
+template <int D, bool TOKQ>
 __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __restrict__ q,
                                                                  const uint4* __restrict__ k,
                                                                  const uint4* __restrict__ v, int N, int Npad,
@@ -103,24 +104,46 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
 #pragma unroll
     for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[u]));
   }
-  amax = block_max(amax, red);   // also orders the vamax_s initialisation and the K staging
+  amax = block_max(amax, red);   // also orders the vamax_s initialisation and the K staging (and is
+                                 // the block absmax of Q for the per-block scale)
   {
     const int c0 = (threadIdx.x % V8) * 8;
 #pragma unroll
     for (int u = 0; u < 8; ++u) atomicMax(&vamax_s[c0 + u], __float_as_int(va[u]));
   }
-  const float qinv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-  if (threadIdx.x == 0) q_scale[(size_t)bh * nK + kb] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
   uint2* qo = reinterpret_cast<uint2*>(q_i8 + ((size_t)bh * Npad + n0) * D);
+  if constexpr (!TOKQ) {
+    const float qinv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+    if (threadIdx.x == 0) q_scale[(size_t)bh * nK + kb] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
 #pragma unroll
-  for (int i = 0; i < PER_T; ++i) {
-    const int e = threadIdx.x + i * kThreads;
-    float x[8];
-    unpack8(qv[i], x);
-    int c[8];
+    for (int i = 0; i < PER_T; ++i) {
+      const int e = threadIdx.x + i * kThreads;
+      float x[8];
+      unpack8(qv[i], x);
+      int c[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) c[u] = qinv > 0.f ? quant_i8(x[u], qinv) : 0;
-    qo[e] = pack_i8x8(c);   // rows >= nr hold zeros (qv was zeroed)
+      for (int u = 0; u < 8; ++u) c[u] = qinv > 0.f ? quant_i8(x[u], qinv) : 0;
+      qo[e] = pack_i8x8(c);   // rows >= nr hold zeros (qv was zeroed)
+    }
+  } else {
+    // the V8 consecutive lanes that hold one token reduce its absmax
+#pragma unroll
+    for (int i = 0; i < PER_T; ++i) {
+      const int e = threadIdx.x + i * kThreads;
+      float x[8];
+      unpack8(qv[i], x);
+      float ra = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ra = fmaxf(ra, fabsf(x[u]));
+#pragma unroll
+      for (int o = V8 / 2; o > 0; o >>= 1) ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, o));
+      const float rinv = ra > 0.f ? __fdiv_rn(127.0f, ra) : 0.f;
+      if (e % V8 == 0) q_scale[(size_t)bh * Npad + n0 + e / V8] = ra > 0.f ? __fdiv_rn(ra, 127.0f) : 0.f;
+      int c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) c[u] = rinv > 0.f ? quant_i8(x[u], rinv) : 0;
+      qo[e] = pack_i8x8(c);   // rows >= nr: zero codes and scale 0
+    }
   }
   __syncthreads();
 
@@ -248,12 +271,17 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
 template <int D>
 cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH, int N, int8_t* q_i8,
                              float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
-                             float* v_scale, const PrepassScratch& scr, cudaStream_t stream) {
+                             float* v_scale, const PrepassScratch& scr, bool q_per_token, cudaStream_t stream) {
   const int nK = num_tiles(N), Npad = nK * kTile;
   dim3 grid(nK, BH);
-  prepass_stats_kernel<D><<<grid, kThreads, 0, stream>>>(
-      static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
-      q_scale, scr);
+  if (q_per_token)
+    prepass_stats_kernel<D, true><<<grid, kThreads, 0, stream>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
+        q_scale, scr);
+  else
+    prepass_stats_kernel<D, false><<<grid, kThreads, 0, stream>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
+        q_scale, scr);
   prepass_finalize_kernel<D><<<BH, D, 0, stream>>>(N, nK, scr, k_mean, v_scale);
   prepass_quant_kv_kernel<D><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(k),
                                                             static_cast<const uint4*>(v), N, Npad, k_mean, k_i8,
@@ -286,13 +314,13 @@ PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d) {
 
 cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
                            float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
-                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream) {
+                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream, bool q_per_token) {
   if (d == 128)
     return launch_prepass_d<128>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
-                                 stream);
+                                 q_per_token, stream);
   if (d == 64)
     return launch_prepass_d<64>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
-                                stream);
+                                q_per_token, stream);
   return cudaErrorInvalidValue;
 }
 

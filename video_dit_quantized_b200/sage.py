@@ -15,6 +15,7 @@ from . import build as _build
 
 MODE_BF16 = 0
 MODE_INT8_FP8 = 1
+MODE_INT8_FP8_QTOKEN = 2
 BLK = 128
 P_SCALE = 448.0
 
@@ -51,6 +52,8 @@ def _load() -> ctypes.CDLL:
         "sage_dbg_attn_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
         "sage_quantize_qk_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
         "sage_attn_fwd_host": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, i32, vp]),
+        "sage_quantize_qk_ex": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sage_attn_quantized_ex": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
         "sage_error_scratch_bytes": (sz, [i32, i32]),
         "sage_attn_error_stats": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
         "sage_select_full_precision_layers": (i32, [vp, i32, i32, ctypes.c_double, vp, vp]),
@@ -116,15 +119,18 @@ def alloc_workspace(B: int, H: int, N: int, d: int, mode: int, device=None):
     return ws
 
 
-def quantize_qk(q, k, v, stream=None):
-    """Runs the prepass; returns a dict of device tensors (q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale)."""
+def quantize_qk(q, k, v, stream=None, q_per_token: bool = False):
+    """Runs the prepass; returns a dict of device tensors (q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale).
+
+    q_per_token: one Q scale per token (q_scale [B,H,nT*128]) instead of per 128-token block.
+    """
     import torch
     B, H, N, d = _bhnd(q, "q")
     dev = q.device
     nT = (N + BLK - 1) // BLK
     out = dict(
         q_i8=torch.empty((B, H, nT * BLK, d), dtype=torch.int8, device=dev),
-        q_scale=torch.empty((B, H, nT), dtype=torch.float32, device=dev),
+        q_scale=torch.empty((B, H, nT * BLK if q_per_token else nT), dtype=torch.float32, device=dev),
         k_i8=torch.empty((B, H, nT * BLK, d), dtype=torch.int8, device=dev),
         k_scale=torch.empty((B, H, nT), dtype=torch.float32, device=dev),
         k_mean=torch.empty((B, H, d), dtype=torch.float32, device=dev),
@@ -133,11 +139,12 @@ def quantize_qk(q, k, v, stream=None):
     )
     nscr = prepass_scratch_bytes(B, H, N, d)
     scratch = torch.empty(max(nscr, 256), dtype=torch.uint8, device=dev)
-    _check(LIB.sage_quantize_qk(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(out["q_i8"]), _ptr(out["q_scale"]),
-                                _ptr(out["k_i8"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]), _ptr(out["v_f8t"]),
-                                _ptr(out["v_scale"]), _ptr(scratch), scratch.numel(), _stream(stream)),
-           "sage_quantize_qk")
+    _check(LIB.sage_quantize_qk_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, 1 if q_per_token else BLK,
+                                   _ptr(out["q_i8"]), _ptr(out["q_scale"]), _ptr(out["k_i8"]), _ptr(out["k_scale"]),
+                                   _ptr(out["k_mean"]), _ptr(out["v_f8t"]), _ptr(out["v_scale"]), _ptr(scratch),
+                                   scratch.numel(), _stream(stream)), "sage_quantize_qk_ex")
     out["_scratch"] = scratch
+    out["_q_per_token"] = bool(q_per_token)
     return out
 
 
@@ -164,9 +171,10 @@ def attn_quantized(pre: dict, N: int, o=None, status=None, stream=None):
         o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=pre["q_i8"].device)
     if status is None:
         status = torch.zeros(64, dtype=torch.int32, device=o.device)
-    _check(LIB.sage_attn_quantized(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]), _ptr(pre["k_scale"]),
-                                   _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o), B, H, N, d, _ptr(status),
-                                   _stream(stream)), "sage_attn_quantized")
+    gran = 1 if pre.get("_q_per_token", False) else BLK
+    _check(LIB.sage_attn_quantized_ex(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]),
+                                      _ptr(pre["k_scale"]), _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o), B, H, N,
+                                      d, gran, _ptr(status), _stream(stream)), "sage_attn_quantized_ex")
     return o
 
 
