@@ -73,6 +73,8 @@ def _load():
             lib.orc_attn_exact.argtypes = [u16, u16, u16, i32, i32, i32, i32, P(i32), i32, f64]
             lib.orc_attn_emul.argtypes = [i8, f32, i8, f32, u8, f32, i32, i32, i32, i32, P(i32), i32, i32,
                                           u16, u16, u16, f32, u16]
+            lib.orc_quant_blocks_2d.argtypes = [u16, i32, i32, i8, f32]
+            lib.orc_linear_w8a8.argtypes = [i8, f32, i8, f32, u16, i32, i32, i32, P(i32), i32, f32, u16]
             lib.orc_layer_schedule.argtypes = [i32, P(i32), i32, i8]
             lib.orc_layer_schedule.restype = i32
             _lib = lib
@@ -203,6 +205,33 @@ def attn_emul(pre: dict, rows=None, flags: int = 0, q=None, k=None, v=None):
                           _p(qb_, ctypes.c_uint16), _p(kb_, ctypes.c_uint16), _p(vb_, ctypes.c_uint16),
                           _p(out, ctypes.c_float), _p(outb, ctypes.c_uint16))
     return out, outb
+
+
+def quant_blocks_2d(x: np.ndarray):
+    """W8A8 operand: INT8 codes [R, K] and fp32 scales [ceil(R/128), K/128] of a bf16 [R, K] matrix."""
+    x = _c(x, np.uint16)
+    R, K = x.shape
+    assert K % 128 == 0
+    codes = np.empty((R, K), dtype=np.int8)
+    scales = np.empty(((R + 127) // 128, K // 128), dtype=np.float32)
+    _load().orc_quant_blocks_2d(_p(x, ctypes.c_uint16), R, K, _p(codes, ctypes.c_int8), _p(scales, ctypes.c_float))
+    return codes, scales
+
+
+def linear_w8a8(xq, sx, wq, sw, bias=None, rows=None):
+    """Y = block-scaled INT8 product (+ bias) for the given rows: (fp32 [R, N], bf16 bits [R, N])."""
+    xq, wq = _c(xq, np.int8), _c(wq, np.int8)
+    sx, sw = _c(sx, np.float32), _c(sw, np.float32)
+    M, K = xq.shape
+    N = wq.shape[0]
+    rows = np.arange(M, dtype=np.int32) if rows is None else _c(np.asarray(rows, dtype=np.int32), np.int32)
+    y = np.empty((len(rows), N), dtype=np.float32)
+    yb = np.empty((len(rows), N), dtype=np.uint16)
+    b = None if bias is None else _c(bias, np.uint16)
+    _load().orc_linear_w8a8(_p(xq, ctypes.c_int8), _p(sx, ctypes.c_float), _p(wq, ctypes.c_int8),
+                            _p(sw, ctypes.c_float), _p(b, ctypes.c_uint16), M, N, K, _p(rows, ctypes.c_int),
+                            len(rows), _p(y, ctypes.c_float), _p(yb, ctypes.c_uint16))
+    return y, yb
 
 
 def layer_schedule(num_layers: int, fp_layers) -> np.ndarray:

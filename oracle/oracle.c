@@ -406,6 +406,74 @@ void orc_attn_emul(const int8_t* q8, const float* q_scale, const int8_t* k8, con
     }
 }
 
+/* ---------------- W8A8 linear with 128x128 block scales ---------------- */
+
+/*
+ * Page 1 of the TMAP write-up, "FFN performance optimisation / linear layer
+ * quantization": linear-layer weights and activations in 8 bits with a
+ * 128 x 128 per-block quantization operator.  Reading: a bf16 matrix
+ * X [R, K] (K a multiple of 128) is cut into 128 x 128 blocks; per block
+ * scale = fl(amax / 127), code = clamp(rne(x * fl(127 / amax)), +-127), the
+ * zero guard of the attention prepass.  codes int8 [R, K]; scales fp32
+ * [ceil(R/128), K/128].
+ */
+void orc_quant_blocks_2d(const uint16_t* x, int R, int K, int8_t* codes, float* scales) {
+    int nr = (R + 127) / 128, nk = K / 128;
+#pragma omp parallel for schedule(static)
+    for (long blk = 0; blk < (long)nr * nk; ++blk) {
+        int rb = (int)(blk / nk), kb = (int)(blk % nk);
+        int r0 = rb * 128, r1 = r0 + 128 < R ? r0 + 128 : R;
+        float amax = 0.0f;
+        for (int r = r0; r < r1; ++r)
+            for (int c = kb * 128; c < kb * 128 + 128; ++c) {
+                float a = fabsf(bf16f(x[(long)r * K + c]));
+                if (a > amax) amax = a;
+            }
+        if (amax == 0.0f) {
+            scales[blk] = 0.0f;
+            for (int r = r0; r < r1; ++r) memset(codes + (long)r * K + kb * 128, 0, 128);
+            continue;
+        }
+        float inv = 127.0f / amax;
+        scales[blk] = amax / 127.0f;
+        for (int r = r0; r < r1; ++r)
+            for (int c = kb * 128; c < kb * 128 + 128; ++c) {
+                double q = rne((double)(bf16f(x[(long)r * K + c]) * inv));
+                if (q > 127.0) q = 127.0;
+                if (q < -127.0) q = -127.0;
+                codes[(long)r * K + c] = (int8_t)q;
+            }
+    }
+}
+
+/*
+ * Y[m, n] = sum over K blocks kb (ascending) of
+ *           fl(sx[m/128, kb] * sw[n/128, kb]) * S_kb[m, n],
+ * S_kb[m, n] = sum_{k in kb} xq[m, k] * wq[n, k] in exact integers, the sum
+ * over kb in fp32; then + bias[n] (bf16, may be NULL), rounded to bf16.
+ * xq [M, K], wq [N, K] int8; sx [ceil(M/128), K/128]; sw [ceil(N/128), K/128];
+ * only the rows in `rows` (n_rows entries) are computed: y fp32 [n_rows, N]
+ * and, if y_bf16, the bf16 bits.
+ */
+void orc_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const uint16_t* bias,
+                     int M, int N, int K, const int* rows, int n_rows, float* y, uint16_t* y_bf16) {
+    int nk = K / 128;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long w = 0; w < (long)n_rows * N; ++w) {
+        int m = rows[w / N], n = (int)(w % N);
+        float acc = 0.0f;
+        for (int kb = 0; kb < nk; ++kb) {
+            int64_t s = 0;
+            for (int k = kb * 128; k < kb * 128 + 128; ++k) s += (int64_t)xq[(long)m * K + k] * wq[(long)n * K + k];
+            float sc = sx[(long)(m / 128) * nk + kb] * sw[(long)(n / 128) * nk + kb];
+            acc = acc + sc * (float)s;
+        }
+        if (bias) acc = acc + bf16f(bias[n]);
+        y[w] = acc;
+        if (y_bf16) y_bf16[w] = f32_bf16_rne(acc);
+    }
+}
+
 /* ---------------- a11: layer schedule ---------------- */
 
 /*
