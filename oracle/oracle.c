@@ -449,8 +449,11 @@ void orc_quant_blocks_2d(const uint16_t* x, int R, int K, int8_t* codes, float* 
 /*
  * Y[m, n] = sum over K blocks kb (ascending) of
  *           fl(sx[m/128, kb] * sw[n/128, kb]) * S_kb[m, n],
- * S_kb[m, n] = sum_{k in kb} xq[m, k] * wq[n, k] in exact integers, the sum
- * over kb in fp32; then + bias[n] (bf16, may be NULL), rounded to bf16.
+ * S_kb[m, n] = sum_{k in kb} xq[m, k] * wq[n, k] in exact integers (|S| <
+ * 2^21, so exact in fp32 too); the sum over kb in fp32, each block's term
+ * added with one fused multiply-add (one rounding: the page fixes no
+ * rounding, a fused multiply-add is the plain fp32 "acc += scale * S");
+ * then + bias[n] (bf16, may be NULL) in fp32, rounded to bf16.
  * xq [M, K], wq [N, K] int8; sx [ceil(M/128), K/128]; sw [ceil(N/128), K/128];
  * only the rows in `rows` (n_rows entries) are computed: y fp32 [n_rows, N]
  * and, if y_bf16, the bf16 bits.
@@ -466,7 +469,7 @@ void orc_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const 
             int64_t s = 0;
             for (int k = kb * 128; k < kb * 128 + 128; ++k) s += (int64_t)xq[(long)m * K + k] * wq[(long)n * K + k];
             float sc = sx[(long)(m / 128) * nk + kb] * sw[(long)(n / 128) * nk + kb];
-            acc = acc + sc * (float)s;
+            acc = fmaf(sc, (float)s, acc);          /* one rounding per block */
         }
         if (bias) acc = acc + bf16f(bias[n]);
         y[w] = acc;

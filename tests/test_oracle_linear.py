@@ -17,6 +17,15 @@ def f(b):
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def f32_rne(r: Fraction) -> np.float32:
+    """The fp32 nearest to the rational r, ties to even (no double rounding through float64)."""
+    c = np.float32(float(r))
+    cands = [c, np.nextafter(c, np.float32(np.inf)), np.nextafter(c, np.float32(-np.inf))]
+    best = min(abs(Fraction(float(x)) - r) for x in cands)
+    near = [x for x in cands if abs(Fraction(float(x)) - r) == best]
+    return min(near, key=lambda x: int(np.array(x).view(np.uint32)) & 1)
+
+
 def test_block_quantizer_matches_the_attention_one_per_block():
     rng = np.random.default_rng(0)
     x = bf16(rng.standard_normal((300, 256)).astype(np.float32) * 2)
@@ -50,8 +59,9 @@ def test_linear_is_the_exact_block_scaled_sum():
             for kb in range(2):
                 s = int(np.dot(xq[m, kb * 128:(kb + 1) * 128].astype(np.int64), wq[n, kb * 128:(kb + 1) * 128].astype(np.int64)))
                 sc = np.float32(sx[m // 128, kb]) * np.float32(sw[n // 128, kb])
-                acc = np.float32(acc + np.float32(sc * np.float32(s)))
-            acc = np.float32(acc + np.float32(f(b[n:n + 1])[0]))
+                # fused multiply-add: the exact rational sc * s + acc, rounded once to fp32
+                acc = f32_rne(Fraction(float(sc)) * s + Fraction(float(acc)))
+            acc = f32_rne(Fraction(float(acc)) + Fraction(float(f(b[n:n + 1])[0])))
             assert y[i, n] == acc
     # and it approximates the exact bf16 product within the INT8 quantization error
     exact = f(x)[rows] @ f(w).T + f(b)
