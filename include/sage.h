@@ -223,6 +223,44 @@ int sage_select_full_precision_layers(const double* layer_err, int num_layers, i
                                       double threshold, int* layers_out, int* n_out);
 
 /*
+ * 8-bit linear layers with 128 x 128 block scales (TMAP write-up, "FFN
+ * performance optimisation / linear-layer quantization": the DiT's linear
+ * weights and activations in 8 bits -- W8A8 -- with a 128 x 128 per-block
+ * quantization operator).  The 8-bit format is symmetric INT8, as in the
+ * attention prepass: per block, scale = amax / 127 and
+ * code = clamp(rne(x * (127 / amax)), -127, 127); an all-zero block gets
+ * scale 0 and codes 0.
+ *
+ * sage_quantize_blocks_2d: x device bf16 [R, K] row-major (R >= 1, K a
+ * positive multiple of 128, ceil(R/128) <= 65535); codes device int8 [R, K];
+ * scales device fp32 [ceil(R/128), K/128], scales[rb][kb] for rows
+ * 128*rb .. +127 (only the real ones) and columns 128*kb .. +127.  Used for
+ * the activations X [M, K] (rows = tokens) and, once, for the weights
+ * W [N, K] (rows = output features).
+ *
+ * sage_linear_w8a8: Y = X W^T + bias from the block-quantized operands:
+ *   Y[m, n] = sum over kb = 0 .. K/128-1 (in that order) of
+ *             fl(sx[m/128][kb] * sw[n/128][kb]) * S_kb[m, n],
+ *   S_kb[m, n] = sum over k in block kb of xq[m, k] * wq[n, k] (exact int32),
+ * the sum over kb in fp32 with one fused multiply-add per block, then
+ * + bias[n] in fp32 and, for y_dtype SAGE_DTYPE_BF16, rounded to bf16 (RNE).
+ *   xq int8 [M, K], sx fp32 [ceil(M/128), K/128]  (sage_quantize_blocks_2d of X)
+ *   wq int8 [N, K], sw fp32 [N/128, K/128]        (sage_quantize_blocks_2d of W)
+ *   bias bf16 [N] or NULL; y [M, N] bf16 or fp32 (y_dtype).
+ * M >= 1; N and K positive multiples of 128.  xq, wq, bias, y 16-byte
+ * aligned; sx, sw 4-byte aligned.  status: device memory whose first uint32
+ * is the status word (the workspace of the attention calls serves);
+ * sage_status() on it reports a bounded wait that ran out.  Asynchronous on
+ * `stream`.
+ */
+#define SAGE_LIN_BLK 128
+#define SAGE_DTYPE_BF16 0
+#define SAGE_DTYPE_F32 1
+int sage_quantize_blocks_2d(const void* x, int R, int K, int8_t* codes, float* scales, void* stream);
+int sage_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias,
+                     void* y, int y_dtype, int M, int N, int K, void* status, void* stream);
+
+/*
  * Reads and clears the device status word at the start of `workspace`
  * (synchronises `stream`).  Returns SAGE_OK, SAGE_ETIMEOUT if a bounded
  * device-side wait ran out since the last call, or SAGE_ELAUNCH if the stream
@@ -275,6 +313,16 @@ int sage_dbg_attn_forced_timeout(const int8_t* q_i8, const float* q_scale, const
                                  const float* k_scale, const uint8_t* v_f8t, const float* v_scale,
                                  void* o, int B, int H, int N, int d, void* status,
                                  long long timeout_cycles, void* stream);
+
+/*
+ * Test hook of the bounded-wait machinery of sage_linear_w8a8: the MMA
+ * thread first waits on a barrier that no one completes, with a wait limit of
+ * `timeout_cycles` SM clocks, so the kernel records SAGE_ETIMEOUT in `status`
+ * and returns without hanging.  Same operands as sage_linear_w8a8.
+ */
+int sage_dbg_linear_forced_timeout(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                                   const void* bias, void* y, int y_dtype, int M, int N, int K, void* status,
+                                   long long timeout_cycles, void* stream);
 
 #ifdef __cplusplus
 }

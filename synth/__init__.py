@@ -52,6 +52,8 @@ def _load():
             lib.synth_sample_rows.restype = i32
             lib.synth_outlier_pairs.argtypes = [u64, i32, i32, i32, ctypes.POINTER(ctypes.c_uint8)]
             lib.synth_outlier_pairs.restype = i32
+            lib.synth_linear.argtypes = [u64, i32, i32, i32, i32, dbl, p16, p16, p16]
+            lib.synth_linear.restype = i32
             lib.synth_normal.argtypes = [u64, ctypes.c_uint32, u64]
             lib.synth_normal.restype = dbl
             _lib = lib
@@ -152,3 +154,54 @@ def outlier_pairs(w: Workload) -> np.ndarray:
 def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
     """Widens bf16 bit patterns (uint16) to float32 exactly."""
     return (a.astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclass(frozen=True)
+class LinearWorkload:
+    """One synthetic linear layer Y = X W^T + bias: X [M, K], W [N, K]."""
+    name: str
+    M: int
+    N: int
+    K: int
+    seed: int = 0
+    outlier_frac: float = 0.01      # fraction of X channels scaled as outliers
+    outlier_scale: float = 20.0
+
+    @property
+    def n_outlier(self) -> int:
+        return int(math.floor(self.outlier_frac * self.K + 0.5))
+
+    @property
+    def flops(self) -> float:
+        """GEMM FLOPs of one call: 2 * M * N * K."""
+        return 2.0 * self.M * self.N * float(self.K)
+
+
+# Wan2.1-14B (hidden 5120, FFN 13824) over the 720p video's 75600 tokens, and
+# small ragged cases (M not a multiple of 128, N an odd multiple of 128).
+LINEAR_WORKLOADS = {
+    "lin_tiny": LinearWorkload("lin_tiny", 333, 384, 512, seed=1),
+    "lin_multi": LinearWorkload("lin_multi", 8197, 1280, 1024, seed=2),
+    "wan14b_720p_proj": LinearWorkload("wan14b_720p_proj", 75600, 5120, 5120, seed=0),
+    "wan14b_720p_ffn_up": LinearWorkload("wan14b_720p_ffn_up", 75600, 13824, 5120, seed=0),
+    "wan14b_720p_ffn_down": LinearWorkload("wan14b_720p_ffn_down", 75600, 5120, 13824, seed=0),
+}
+
+
+def linear_numpy(w: LinearWorkload, parts: str = "xwb"):
+    """Returns (x [M, K], w [N, K], bias [N]) as uint16 arrays of bf16 bits."""
+    lib = _load()
+    out = {
+        "x": np.empty((w.M, w.K), dtype=np.uint16) if "x" in parts else None,
+        "w": np.empty((w.N, w.K), dtype=np.uint16) if "w" in parts else None,
+        "b": np.empty((w.N,), dtype=np.uint16) if "b" in parts else None,
+    }
+
+    def ptr(a):
+        return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)) if a is not None else None
+
+    rc = lib.synth_linear(w.seed, w.M, w.N, w.K, w.n_outlier, w.outlier_scale, ptr(out["x"]), ptr(out["w"]),
+                          ptr(out["b"]))
+    if rc != 0:
+        raise ValueError(f"synth_linear rejected workload {w}")
+    return out["x"], out["w"], out["b"]

@@ -33,6 +33,10 @@
 #define SYN_KOFF 4u
 #define SYN_OUTLIER 5u
 #define SYN_ROWS 6u
+#define SYN_LX 7u
+#define SYN_LW 8u
+#define SYN_LB 9u
+#define SYN_LOUT 10u
 
 static inline uint64_t splitmix64(uint64_t x) {
     x += 0x9E3779B97F4A7C15ull;
@@ -70,11 +74,11 @@ double synth_normal(uint64_t seed, uint32_t tensor, uint64_t e) {
 }
 
 /* Marks the outlier (h, c) pairs: the n_out pairs with the smallest hash. */
-static void outlier_mask(uint64_t seed, int H, int d, int n_out, uint8_t* mask) {
+static void outlier_mask_t(uint64_t seed, uint32_t tensor, int H, int d, int n_out, uint8_t* mask) {
     int total = H * d;
     memset(mask, 0, (size_t)total);
     if (n_out <= 0) return;
-    uint64_t key = stream_key(seed, SYN_OUTLIER);
+    uint64_t key = stream_key(seed, tensor);
     uint64_t* h = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)total);
     for (int i = 0; i < total; ++i) h[i] = splitmix64(key + (uint64_t)i);
     for (int k = 0; k < n_out && k < total; ++k) {
@@ -84,6 +88,10 @@ static void outlier_mask(uint64_t seed, int H, int d, int n_out, uint8_t* mask) 
         mask[best] = 1;
     }
     free(h);
+}
+
+static void outlier_mask(uint64_t seed, int H, int d, int n_out, uint8_t* mask) {
+    outlier_mask_t(seed, SYN_OUTLIER, H, d, n_out, mask);
 }
 
 int synth_outlier_pairs(uint64_t seed, int H, int d, int n_out, uint8_t* mask_out) {
@@ -163,4 +171,41 @@ int synth_sample_rows(uint64_t seed, int N, int n, int* rows) {
     free(taken);
     qsort(rows, (size_t)cnt, sizeof(int), cmp_int);
     return cnt;
+}
+
+/*
+ * Linear-layer operands, bf16 bit patterns, row-major:
+ *   x [M, K]  N(0,1), the n_outlier channels k with the smallest hash scaled
+ *             by outlier_scale (activation outlier channels)
+ *   w [N, K]  N(0,1) / sqrt(K)
+ *   bias [N]  0.02 * N(0,1)
+ * Any pointer may be NULL to skip that tensor.
+ */
+int synth_linear(uint64_t seed, int M, int N, int K, int n_outlier, double outlier_scale,
+                 uint16_t* x, uint16_t* w, uint16_t* bias) {
+    if (M <= 0 || N <= 0 || K <= 0 || n_outlier < 0 || n_outlier > K) return -1;
+    uint8_t* mask = (uint8_t*)malloc((size_t)K);
+    outlier_mask_t(seed, SYN_LOUT, 1, K, n_outlier, mask);
+    const uint64_t kx = stream_key(seed, SYN_LX), kw = stream_key(seed, SYN_LW), kb = stream_key(seed, SYN_LB);
+    const double wstd = 1.0 / sqrt((double)K);
+    if (x) {
+#pragma omp parallel for schedule(static)
+        for (long r = 0; r < (long)M; ++r)
+            for (int c = 0; c < K; ++c) {
+                uint64_t e = (uint64_t)r * (uint64_t)K + (uint64_t)c;
+                x[e] = f32_to_bf16((float)(normal_at(kx, e) * (mask[c] ? outlier_scale : 1.0)));
+            }
+    }
+    if (w) {
+#pragma omp parallel for schedule(static)
+        for (long r = 0; r < (long)N; ++r)
+            for (int c = 0; c < K; ++c) {
+                uint64_t e = (uint64_t)r * (uint64_t)K + (uint64_t)c;
+                w[e] = f32_to_bf16((float)(normal_at(kw, e) * wstd));
+            }
+    }
+    if (bias)
+        for (int n = 0; n < N; ++n) bias[n] = f32_to_bf16((float)(0.02 * normal_at(kb, (uint64_t)n)));
+    free(mask);
+    return 0;
 }

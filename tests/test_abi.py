@@ -12,6 +12,7 @@ EXPECTED = {
     "sage_dbg_qk_tiles", "sage_dbg_pv_tile", "sage_dbg_qk_bf16_tile", "sage_dbg_attn_forced_timeout",
     "sage_quantize_qk_noalloc", "sage_attn_fwd_host", "sage_error_scratch_bytes", "sage_attn_error_stats",
     "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
+    "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
 }
 
 
@@ -77,3 +78,34 @@ def test_select_full_precision_layers_host():
     assert sage.select_full_precision_layers(err, 1.0) == []
     with pytest.raises(sage.SageError):
         sage.select_full_precision_layers([[float("nan")]], 0.1)
+
+
+def test_linear_argument_validation_runs_on_the_host():
+    """Bad sizes and pointers are refused before any device call (works without a GPU)."""
+    lib = sage.LIB
+    fake = ctypes.c_void_p(1 << 20)            # 16-byte aligned, never dereferenced on these paths
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    s = None
+    args = lambda **kw: [kw.get("xq", fake), kw.get("sx", fake), kw.get("wq", fake), kw.get("sw", fake),
+                         kw.get("bias", None), kw.get("y", fake), kw.get("dt", sage.DTYPE_BF16), kw.get("M", 256),
+                         kw.get("N", 256), kw.get("K", 256), kw.get("st", fake), s]
+    assert lib.sage_linear_w8a8(*args(N=200)) == sage.EINVAL        # N not a multiple of 128
+    assert lib.sage_linear_w8a8(*args(K=64)) == sage.EINVAL         # K below one block
+    assert lib.sage_linear_w8a8(*args(M=0)) == sage.EINVAL
+    assert lib.sage_linear_w8a8(*args(dt=7)) == sage.EINVAL
+    assert lib.sage_linear_w8a8(*args(xq=None)) == sage.EINVAL
+    assert lib.sage_linear_w8a8(*args(y=odd)) == sage.EINVAL        # misaligned output
+    assert lib.sage_linear_w8a8(*args(bias=odd)) == sage.EINVAL
+    assert lib.sage_dbg_linear_forced_timeout(*args()[:11], 0, s) == sage.EINVAL
+    assert lib.sage_quantize_blocks_2d(fake, 100, 130, fake, fake, s) == sage.EINVAL
+    assert lib.sage_quantize_blocks_2d(fake, 0, 128, fake, fake, s) == sage.EINVAL
+    assert lib.sage_quantize_blocks_2d(fake, 128 * 65536, 128, fake, fake, s) == sage.EINVAL
+    assert lib.sage_quantize_blocks_2d(odd, 100, 128, fake, fake, s) == sage.EINVAL
+    if not _has_gpu():
+        # well-formed arguments reach the device check, which reports no usable device
+        assert lib.sage_linear_w8a8(*args()) in (sage.ELAUNCH, sage.EUNSUPPORTED)
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()

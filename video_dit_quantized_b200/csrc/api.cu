@@ -291,6 +291,52 @@ int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_
   return SAGE_OK;
 }
 
+namespace {
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_linear(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
+                 int y_dtype, int M, int N, int K, void* status) {
+  if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return SAGE_EINVAL;
+  if (y_dtype != SAGE_DTYPE_BF16 && y_dtype != SAGE_DTYPE_F32) return SAGE_EINVAL;
+  const void* p16[] = {xq, wq, y};
+  for (const void* p : p16)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if (bias && !aligned16(bias)) return SAGE_EINVAL;
+  const void* p4[] = {sx, sw, status};
+  for (const void* p : p4)
+    if (!p || !aligned4(p)) return SAGE_EINVAL;
+  return check_device();
+}
+}  // namespace
+
+int sage_quantize_blocks_2d(const void* x, int R, int K, int8_t* codes, float* scales, void* stream) {
+  if (R < 1 || K < 128 || K % 128 != 0 || (R + 127) / 128 > 65535) return SAGE_EINVAL;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes) || !aligned4(scales)) return SAGE_EINVAL;
+  const int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_quant_blocks_2d(x, R, K, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
+                     int y_dtype, int M, int N, int K, void* status, void* stream) {
+  const int rc = check_linear(xq, sx, wq, sw, bias, y, y_dtype, M, N, K, status);
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_linear_w8a8(xq, sx, wq, sw, bias, y, y_dtype == SAGE_DTYPE_F32, M, N, K,
+                                          static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int sage_dbg_linear_forced_timeout(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                                   const void* bias, void* y, int y_dtype, int M, int N, int K, void* status,
+                                   long long timeout_cycles, void* stream) {
+  if (timeout_cycles < 1) return SAGE_EINVAL;
+  const int rc = check_linear(xq, sx, wq, sw, bias, y, y_dtype, M, N, K, status);
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_linear_w8a8(xq, sx, wq, sw, bias, y, y_dtype == SAGE_DTYPE_F32, M, N, K,
+                                          static_cast<uint32_t*>(status), timeout_cycles, 1,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int sage_status(void* workspace, void* stream) {
   if (!workspace) return SAGE_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -44,6 +44,12 @@ cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N, int d,
                              uint32_t* status, long long timeout_cycles, cudaStream_t stream);
 
+// 8-bit linear layers with 128 x 128 block scales.
+cudaError_t launch_quant_blocks_2d(const void* x, int R, int K, int8_t* codes, float* scales, cudaStream_t stream);
+cudaError_t launch_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias,
+                               void* y, int y_f32, int M, int N, int K, uint32_t* status, long long timeout_cycles,
+                               int dbg_flags, cudaStream_t stream);
+
 // Diagnostics.
 cudaError_t launch_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int BH, int H, int N, int d,
                                 const int* tile_list, int n, int32_t* out, cudaStream_t stream);

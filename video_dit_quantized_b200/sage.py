@@ -16,6 +16,8 @@ from . import build as _build
 MODE_BF16 = 0
 MODE_INT8_FP8 = 1
 MODE_INT8_FP8_QTOKEN = 2
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
 BLK = 128
 P_SCALE = 448.0
 
@@ -57,6 +59,9 @@ def _load() -> ctypes.CDLL:
         "sage_error_scratch_bytes": (sz, [i32, i32]),
         "sage_attn_error_stats": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
         "sage_select_full_precision_layers": (i32, [vp, i32, i32, ctypes.c_double, vp, vp]),
+        "sage_quantize_blocks_2d": (i32, [vp, i32, i32, vp, vp, vp]),
+        "sage_linear_w8a8": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
+        "sage_dbg_linear_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -258,6 +263,38 @@ def select_full_precision_layers(layer_err, threshold: float) -> list[int]:
     return [int(out[i]) for i in range(n.value)]
 
 
+def quantize_blocks_2d(x, codes=None, scales=None, stream=None):
+    """bf16 [R, K] -> (int8 codes [R, K], fp32 scales [ceil(R/128), K/128]), 128 x 128 blocks."""
+    import torch
+    if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bf16 [R, K] tensor")
+    R, K = x.shape
+    if codes is None:
+        codes = torch.empty((R, K), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(((R + BLK - 1) // BLK, K // BLK), dtype=torch.float32, device=x.device)
+    _check(LIB.sage_quantize_blocks_2d(_ptr(x), R, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "sage_quantize_blocks_2d")
+    return codes, scales
+
+
+def linear_w8a8(xq, sx, wq, sw, bias=None, y=None, out_dtype=None, status=None, stream=None):
+    """Y = X W^T + bias from 128 x 128 block-quantized X [M, K] and W [N, K]; returns Y [M, N]."""
+    import torch
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out_dtype is None:
+        out_dtype = torch.bfloat16 if y is None else y.dtype
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    if status is None:
+        status = torch.zeros(64, dtype=torch.int32, device=xq.device)
+    code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
+    _check(LIB.sage_linear_w8a8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M, N, K,
+                                _ptr(status), _stream(stream)), "sage_linear_w8a8")
+    return y
+
+
 def status(workspace, stream=None) -> int:
     """Reads and clears the device status word (synchronises the stream); returns a status code."""
     return int(LIB.sage_status(_ptr(workspace), _stream(stream)))
@@ -304,6 +341,19 @@ def dbg_qk_bf16_tile(q, k, stream=None):
     out = torch.empty((BLK, BLK), dtype=torch.float32, device=q.device)
     _check(LIB.sage_dbg_qk_bf16_tile(_ptr(q), _ptr(k), d, _ptr(out), _stream(stream)), "sage_dbg_qk_bf16_tile")
     return out
+
+
+def dbg_linear_forced_timeout(xq, sx, wq, sw, status, timeout_cycles: int, bias=None, y=None, stream=None):
+    import torch
+    M, K = xq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
+    _check(LIB.sage_dbg_linear_forced_timeout(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M,
+                                              N, K, _ptr(status), int(timeout_cycles), _stream(stream)),
+           "sage_dbg_linear_forced_timeout")
+    return y
 
 
 def dbg_attn_forced_timeout(pre: dict, N: int, status, timeout_cycles: int, o=None, stream=None):
