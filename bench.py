@@ -9,6 +9,13 @@ HBM.  Metric: attention TFLOPS = 4 * B * H * N^2 * d / step time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME] [--mode int8_fp8|bf16]
+  python bench.py --op linear [--linear-workload NAME]
+
+`--op linear` times the W8A8 linear layer with 128 x 128 block scales
+instead (one step = block-quantize the activations X [M, K] + the block-scaled
+INT8 GEMM against pre-quantized weights W [N, K], plus bias), at the
+Wan2.1-14B 720p projection shape 75600 x 5120 x 5120 by default; metric
+TOPS = 2 * M * N * K / step time.
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 device (independent attention calls; no data-path collective), so scaling is
@@ -46,6 +53,11 @@ NCU_TRAFFIC_BYTES = {
     ("wan14b_720p", 40, "int8_fp8"): 1.653e9,
     ("wan14b_720p", 40, "bf16"): 3.002e9,
 }
+# W8A8 GEMM DRAM bytes per launch (ncu capture of the same kernel, summarised in
+# profiles/linear_w8a8_wan14b_720p.md).  Absent keys report null.
+NCU_TRAFFIC_BYTES_LINEAR = {
+    ("wan14b_720p_proj", "w8a8"): 1.160e9,
+}
 
 
 def parse():
@@ -60,6 +72,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3, help="end-to-end steps (at least 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--op", default="attention", choices=["attention", "linear"])
+    ap.add_argument("--linear-workload", default="wan14b_720p_proj", choices=sorted(synth.LINEAR_WORKLOADS))
     return ap.parse_args()
 
 
@@ -167,8 +181,34 @@ def cpu_baseline(w, n_rows: int, impl_line: bool = False):
             "seconds": dt}
 
 
+def run_reference_linear(args, rank, world):
+    """Reference arm of --op linear: the CPU oracle on a bounded sample per step."""
+    w = synth.LINEAR_WORKLOADS[args.linear_workload]
+    if rank != 0:
+        return
+    vals, secs = [], []
+    for i in range(max(args.warmup, 0) + args.steps):
+        r = cpu_baseline_linear(w, 64 if i < args.warmup else 256)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            secs.append(r["seconds"])
+    tops = statistics.median(vals)
+    print(json.dumps({
+        "impl": "reference", "op": "linear_w8a8", "metric": "W8A8 linear TOPS per call (2*M*N*K)", "value": tops,
+        "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int64 block sums, f32 (CPU oracle)", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "sample": "256 sampled rows per step"},
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": r["cores"], "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def run_reference(args, rank, world):
     """Reference arm: the CPU oracle, timed on the host cores, same metric."""
+    if args.op == "linear":
+        run_reference_linear(args, rank, world)
+        return
     w = workload(args)
     if rank != 0:
         return
@@ -360,6 +400,153 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def cpu_baseline_linear(w, n_rows: int):
+    """The oracle as it stands on a bounded sample: 2-D block quantization of the
+    128-row blocks holding n_rows sampled rows of X, and the block-scaled GEMM
+    of those rows against the (pre-quantized) weights."""
+    import oracle
+    x, wt, b = synth.linear_numpy(w)
+    wq, sw = oracle.quant_blocks_2d(wt)
+    rows = synth.sample_rows(w.seed + 7, w.M, n_rows)
+    blocks = np.unique(rows // 128)
+    t0 = time.perf_counter()
+    xs = np.concatenate([x[r * 128:(r + 1) * 128] for r in blocks])
+    xq, sx = oracle.quant_blocks_2d(xs)
+    local = np.array([np.searchsorted(blocks, r // 128) * 128 + r % 128 for r in rows], dtype=np.int32)
+    oracle.linear_w8a8(xq, sx, wq, sw, b, local)
+    dt = time.perf_counter() - t0
+    ops = 2.0 * len(rows) * w.N * w.K
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"128x128 block quantization of the {len(blocks)} row blocks holding {len(rows)} sampled rows "
+                      f"of X + block-scaled INT8 GEMM of those rows (N={w.N}, K={w.K}); TOPS = 2*rows*N*K/time",
+            "seconds": dt}
+
+
+def run_linear(args, rank, world, local_rank):
+    """W8A8 linear: block-quantize X, block-scaled INT8 GEMM (+ bias) against pre-quantized W."""
+    import torch
+    import torch.distributed as dist
+    from video_dit_quantized_b200 import sage
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.LINEAR_WORKLOADS[args.linear_workload]
+    wr = w if rank == 0 else synth.LinearWorkload(w.name, w.M, w.N, w.K, seed=w.seed + rank,
+                                                  outlier_frac=w.outlier_frac, outlier_scale=w.outlier_scale)
+    x_np, w_np, b_np = synth.linear_numpy(wr)
+    as_bf16 = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    x_h = as_bf16(x_np).pin_memory()
+    x = x_h.to(dev)
+    wt, bias = as_bf16(w_np).to(dev), as_bf16(b_np).to(dev)
+    stream = torch.cuda.current_stream()
+    nk = w.K // 128
+    wq, sw = sage.quantize_blocks_2d(wt)                  # weights: quantized once, outside the step
+    xq = torch.empty((w.M, w.K), dtype=torch.int8, device=dev)
+    sx = torch.empty(((w.M + 127) // 128, nk), dtype=torch.float32, device=dev)
+    y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(64, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    sp = sage._stream(stream)
+    P = sage._ptr
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        rc = sage.LIB.sage_quantize_blocks_2d(P(x), w.M, w.K, P(xq), P(sx), sp)
+        if rc:
+            raise sage.SageError(rc, "sage_quantize_blocks_2d")
+        if ev:
+            ev[1].record(stream)
+        rc = sage.LIB.sage_linear_w8a8(P(xq), P(sx), P(wq), P(sw), P(bias), P(y), sage.DTYPE_BF16, w.M, w.N, w.K,
+                                       P(status), sp)
+        if rc:
+            raise sage.SageError(rc, "sage_linear_w8a8")
+        if ev:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sage.status(status) != sage.OK:
+        raise sage.SageError(sage.ETIMEOUT, "warm-up")
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    quant_ms = [a.elapsed_time(b) for a, b, _ in evs]
+    gemm_ms = [b.elapsed_time(c) for _, b, c in evs]
+    if sage.status(status) != sage.OK:
+        raise sage.SageError(sage.ETIMEOUT, "timed region")
+
+    # end to end through the binding: pinned host X in, bf16 Y out, every step
+    y_h = torch.empty((w.M, w.N), dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        sage.quantize_blocks_2d(x, xq, sx, stream=stream)
+        sage.linear_w8a8(xq, sx, wq, sw, bias, y=y, status=status, stream=stream)
+        y_h.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), world, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_linear(w, 1024)
+        cpu.pop("seconds", None)
+    if rank != 0:
+        return
+    ms_step = total_ms / args.steps
+    peaks, src = load_peaks()
+    peak = 2.0 * float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    gemm_avg = statistics.mean(gemm_ms)
+    achieved = w.flops / (gemm_avg * 1e-3) / 1e12
+    line = {
+        "op": "linear_w8a8",
+        "metric": "W8A8 linear TOPS per call (2*M*N*K)",
+        "value": world * w.flops / (ms_step * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 (int32 block sums, fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "global_batch": world,
+                   "parallelism": f"independent calls x{world}",
+                   "l2": "X (774 MB bf16) larger than L2; no flush"},
+        "kernels_ms": {"quantize_median": statistics.median(quant_ms), "gemm_median": statistics.median(gemm_ms),
+                       "gemm_min": min(gemm_ms), "gemm_max": max(gemm_ms)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": NCU_TRAFFIC_BYTES_LINEAR.get((w.name, "w8a8")),
+                     "peak_basis": f"2x bf16_tflops_sustained ({src})",
+                     "frac_of_datasheet_4500": achieved / 4500.0},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * w.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     args.e2e_steps = max(1, args.e2e_steps)
@@ -378,7 +565,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.op == "linear":
+            run_linear(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
