@@ -70,6 +70,26 @@ def test_linear_bit_exact(name, with_bias, cuda_dev):
     np.testing.assert_array_equal(_bits(y16[ridx]), yb_o)
 
 
+def test_linear_long_k_scale_windows(cuda_dev):
+    """K = 13824 (the FFN-down depth: 108 K blocks, so the per-lane scale windows roll over three
+    times), ragged M and an odd multiple of 128 in N; every output, fp32 and bf16."""
+    import torch
+    from video_dit_quantized_b200 import sage
+    w = synth.LinearWorkload("long_k", 200, 384, 13824, seed=11)
+    x, wt, b, xd, wd, bd = _case(w, cuda_dev)
+    xq, sx = sage.quantize_blocks_2d(xd)
+    wq, sw = sage.quantize_blocks_2d(wd)
+    y32 = sage.linear_w8a8(xq, sx, wq, sw, bd, out_dtype=torch.float32)
+    y16 = sage.linear_w8a8(xq, sx, wq, sw, bd)
+    torch.cuda.synchronize()
+    xq_o, sx_o = oracle.quant_blocks_2d(x)
+    wq_o, sw_o = oracle.quant_blocks_2d(wt)
+    np.testing.assert_array_equal(sx.cpu().numpy().view(np.uint32), sx_o.view(np.uint32))
+    y_o, yb_o = oracle.linear_w8a8(xq_o, sx_o, wq_o, sw_o, b)
+    np.testing.assert_array_equal(y32.cpu().numpy().view(np.uint32), y_o.view(np.uint32))
+    np.testing.assert_array_equal(_bits(y16), yb_o)
+
+
 def test_linear_minimal_shape_and_determinism(cuda_dev):
     import torch
     from video_dit_quantized_b200 import sage
