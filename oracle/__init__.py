@@ -75,6 +75,7 @@ def _load():
                                           u16, u16, u16, f32, u16]
             lib.orc_quant_blocks_2d.argtypes = [u16, i32, i32, i8, f32]
             lib.orc_linear_w8a8.argtypes = [i8, f32, i8, f32, u16, i32, i32, i32, P(i32), i32, f32, u16]
+            lib.orc_dequant_blocks_2d.argtypes = [i8, f32, i32, i32, u16]
             lib.orc_layer_schedule.argtypes = [i32, P(i32), i32, i8]
             lib.orc_layer_schedule.restype = i32
             _lib = lib
@@ -232,6 +233,33 @@ def linear_w8a8(xq, sx, wq, sw, bias=None, rows=None):
                             _p(sw, ctypes.c_float), _p(b, ctypes.c_uint16), M, N, K, _p(rows, ctypes.c_int),
                             len(rows), _p(y, ctypes.c_float), _p(yb, ctypes.c_uint16))
     return y, yb
+
+
+def dequant_blocks_2d(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """bf16 bits [R, K] of the block-scaled codes: bf16_rne(fl(scale * code))."""
+    codes, scales = _c(codes, np.int8), _c(scales, np.float32)
+    R, K = codes.shape
+    out = np.empty((R, K), dtype=np.uint16)
+    _load().orc_dequant_blocks_2d(_p(codes, ctypes.c_int8), _p(scales, ctypes.c_float), R, K,
+                                  _p(out, ctypes.c_uint16))
+    return out
+
+
+def linear_bf16(x: np.ndarray, w: np.ndarray, bias=None, rows=None) -> np.ndarray:
+    """Y = X W^T (+ bias) for bf16 bits X [M, K], W [N, K]: the exact products summed in fp64
+    (a library matmul of the fp64 values), returned in fp64 for the given rows."""
+    X = _bf16_f64(np.asarray(x, dtype=np.uint16))
+    W = _bf16_f64(np.asarray(w, dtype=np.uint16))
+    if rows is not None:
+        X = X[np.asarray(rows)]
+    y = X @ W.T
+    if bias is not None:
+        y = y + _bf16_f64(np.asarray(bias, dtype=np.uint16))[None, :]
+    return y
+
+
+def _bf16_f64(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def layer_schedule(num_layers: int, fp_layers) -> np.ndarray:

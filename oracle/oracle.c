@@ -477,6 +477,22 @@ void orc_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const 
     }
 }
 
+/*
+ * W8A16 weights (TMAP write-up, FFN section: weights kept in 8 bits while
+ * some layers compute with 16-bit activations): the bf16 weight a 16-bit
+ * GEMM consumes is the block-scaled code rounded to bf16,
+ * w[r, k] = bf16_rne(fl(scales[r/128, k/128] * codes[r, k])).
+ */
+void orc_dequant_blocks_2d(const int8_t* codes, const float* scales, int R, int K, uint16_t* out) {
+    int nk = K / 128;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < (long)R; ++r)
+        for (int k = 0; k < K; ++k) {
+            float v = scales[(r / 128) * nk + k / 128] * (float)codes[r * K + k];
+            out[r * K + k] = f32_bf16_rne(v);
+        }
+}
+
 /* ---------------- a11: layer schedule ---------------- */
 
 /*

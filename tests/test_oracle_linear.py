@@ -121,3 +121,40 @@ def test_quantizer_is_rational_rne_on_a_tiny_block():
             want = round(prod)                                    # Python's round is half-to-even
             assert codes[r, c] == max(-127, min(127, want))
     assert amax == 3
+
+
+def test_dequant_closed_form_and_round_trip():
+    # a block whose codes are all +-127 dequantizes to +-amax (scale * 127 = amax up to one fp32 rounding)
+    rng = np.random.default_rng(5)
+    w = bf16(rng.standard_normal((256, 256)).astype(np.float32) * 0.05)
+    codes, scales = oracle.quant_blocks_2d(w)
+    deq = oracle.dequant_blocks_2d(codes, scales)
+    for rb in range(2):
+        for kb in range(2):
+            c = codes[rb * 128:(rb + 1) * 128, kb * 128:(kb + 1) * 128].astype(np.int64)
+            d = f(deq[rb * 128:(rb + 1) * 128, kb * 128:(kb + 1) * 128])
+            sc = np.float32(scales[rb, kb])
+            for cv in (-127, -3, 0, 1, 64, 127):
+                m = c == cv
+                if m.any():
+                    want = f(bf16(np.array([np.float32(sc) * np.float32(cv)], dtype=np.float32)))[0]
+                    assert np.all(d[m] == want)
+    # dequantized weights approximate the originals within half a step plus bf16 rounding
+    W = f(w)
+    S = np.repeat(np.repeat(scales.astype(np.float64), 128, 0), 128, 1)
+    assert np.all(np.abs(f(deq) - W) <= S / 2 + np.abs(W) * 2.0 ** -8 + 1e-12)
+    # all-zero block: zeros
+    z = np.zeros((128, 128), dtype=np.uint16)
+    assert not oracle.dequant_blocks_2d(*oracle.quant_blocks_2d(z)).any()
+
+
+def test_linear_bf16_is_the_exact_product():
+    # small integers: every product and sum is exact, so the fp64 result is exact
+    rng = np.random.default_rng(6)
+    x = bf16(rng.integers(-8, 9, (5, 256)).astype(np.float32))
+    w = bf16(rng.integers(-8, 9, (7, 256)).astype(np.float32))
+    b = bf16(rng.integers(-8, 9, 7).astype(np.float32))
+    y = oracle.linear_bf16(x, w, b)
+    X, W, B = (f(a).astype(np.int64) for a in (x, w, b))
+    assert np.array_equal(y, (X @ W.T + B[None, :]).astype(np.float64))
+    assert np.array_equal(oracle.linear_bf16(x, w, None, rows=[4, 0]), (X @ W.T)[[4, 0]].astype(np.float64))
