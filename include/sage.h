@@ -261,6 +261,36 @@ int sage_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const 
                      void* y, int y_dtype, int M, int N, int K, void* status, void* stream);
 
 /*
+ * W8A16 and bf16 linear layers (TMAP write-up, FFN section: to keep video
+ * quality some layers go back from W8A8 to W8A16 -- the weights stay in
+ * 8 bits, the activations and the arithmetic are 16-bit).
+ *
+ * sage_dequant_blocks_2d: out[r][k] = bf16_rne(fl(scales[r/128][k/128] *
+ * codes[r][k])) for codes int8 [R, K] and scales fp32 [ceil(R/128), K/128]
+ * as written by sage_quantize_blocks_2d; out device bf16 [R, K].  K a
+ * positive multiple of 128, ceil(R/128) <= 65535.
+ *
+ * sage_linear_bf16: Y = X W^T + bias with x bf16 [M, K], w bf16 [N, K],
+ * bias bf16 [N] or NULL, y [M, N] bf16 or fp32 (y_dtype); products and sums
+ * in fp32 on the tensor cores (summation order unspecified), bias added in
+ * fp32, bf16 output rounded to nearest even.  M >= 1, N a positive multiple
+ * of 128, K a positive multiple of 64; x, w, bias, y 16-byte aligned.
+ *
+ * sage_linear_w8a16: the W8A16 layer, sage_dequant_blocks_2d of (wq, sw)
+ * into `workspace` followed by sage_linear_bf16 against it.  K a positive
+ * multiple of 128; workspace: device memory of at least
+ * sage_linear_w8a16_workspace_bytes(N, K) bytes, 16-byte aligned.
+ *
+ * status as for sage_linear_w8a8.  Asynchronous on `stream`.
+ */
+int sage_dequant_blocks_2d(const int8_t* codes, const float* scales, int R, int K, void* out, void* stream);
+int sage_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M, int N, int K,
+                     void* status, void* stream);
+size_t sage_linear_w8a16_workspace_bytes(int N, int K);
+int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const void* bias, void* y, int y_dtype,
+                      int M, int N, int K, void* workspace, size_t workspace_bytes, void* status, void* stream);
+
+/*
  * Reads and clears the device status word at the start of `workspace`
  * (synchronises `stream`).  Returns SAGE_OK, SAGE_ETIMEOUT if a bounded
  * device-side wait ran out since the last call, or SAGE_ELAUNCH if the stream

@@ -13,6 +13,7 @@ EXPECTED = {
     "sage_quantize_qk_noalloc", "sage_attn_fwd_host", "sage_error_scratch_bytes", "sage_attn_error_stats",
     "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
     "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
+    "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
 }
 
 
@@ -109,3 +110,17 @@ def test_linear_argument_validation_runs_on_the_host():
 def _has_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+def test_bf16_and_w8a16_argument_validation_runs_on_the_host():
+    lib = sage.LIB
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    s = None
+    assert lib.sage_linear_bf16(fake, fake, None, fake, 0, 256, 256, 96, fake, s) == sage.EINVAL   # K % 64
+    assert lib.sage_linear_bf16(fake, fake, None, fake, 0, 256, 192, 128, fake, s) == sage.EINVAL  # N % 128
+    assert lib.sage_linear_bf16(odd, fake, None, fake, 0, 256, 256, 128, fake, s) == sage.EINVAL
+    assert lib.sage_linear_w8a16_workspace_bytes(256, 384) == 256 * 384 * 2
+    assert lib.sage_linear_w8a16(fake, fake, fake, None, fake, 0, 64, 256, 192, fake, 10 ** 9, fake, s) == sage.EINVAL
+    assert lib.sage_linear_w8a16(fake, fake, fake, None, fake, 0, 64, 256, 256, fake, 1000, fake, s) == sage.EWORKSPACE
+    assert lib.sage_dequant_blocks_2d(fake, fake, 10, 100, fake, s) == sage.EINVAL

@@ -337,6 +337,58 @@ int sage_dbg_linear_forced_timeout(const int8_t* xq, const float* sx, const int8
                                           static_cast<cudaStream_t>(stream)));
 }
 
+int sage_dequant_blocks_2d(const int8_t* codes, const float* scales, int R, int K, void* out, void* stream) {
+  if (R < 1 || K < 128 || K % 128 != 0 || (R + 127) / 128 > 65535) return SAGE_EINVAL;
+  if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) || !aligned4(scales)) return SAGE_EINVAL;
+  const int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_dequant_blocks_2d(codes, scales, R, K, out, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+int check_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M, int N, int K,
+                      void* status) {
+  if (M < 1 || N < 128 || K < 64 || N % 128 != 0 || K % 64 != 0) return SAGE_EINVAL;
+  if (y_dtype != SAGE_DTYPE_BF16 && y_dtype != SAGE_DTYPE_F32) return SAGE_EINVAL;
+  const void* p16[] = {x, w, y};
+  for (const void* p : p16)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if (bias && !aligned16(bias)) return SAGE_EINVAL;
+  if (!status || !aligned4(status)) return SAGE_EINVAL;
+  return SAGE_OK;
+}
+}  // namespace
+
+int sage_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M, int N, int K,
+                     void* status, void* stream) {
+  int rc = check_linear_bf16(x, w, bias, y, y_dtype, M, N, K, status);
+  if (rc != SAGE_OK) return rc;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  return launch_status(launch_linear_bf16(x, w, bias, y, y_dtype == SAGE_DTYPE_F32, M, N, K,
+                                          static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t sage_linear_w8a16_workspace_bytes(int N, int K) {
+  if (N < 1 || K < 1) return 0;
+  return align_up((size_t)N * K * 2, 256);
+}
+
+int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const void* bias, void* y, int y_dtype, int M,
+                      int N, int K, void* workspace, size_t workspace_bytes, void* status, void* stream) {
+  if (K % 128 != 0 || (N + 127) / 128 > 65535) return SAGE_EINVAL;
+  int rc = check_linear_bf16(x, workspace, bias, y, y_dtype, M, N, K, status);
+  if (rc != SAGE_OK) return rc;
+  if (!wq || !sw || !aligned16(wq) || !aligned4(sw)) return SAGE_EINVAL;
+  if (workspace_bytes < sage_linear_w8a16_workspace_bytes(N, K)) return SAGE_EWORKSPACE;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = launch_status(launch_dequant_blocks_2d(wq, sw, N, K, workspace, st));
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_linear_bf16(x, workspace, bias, y, y_dtype == SAGE_DTYPE_F32, M, N, K,
+                                          static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0, st));
+}
+
 int sage_status(void* workspace, void* stream) {
   if (!workspace) return SAGE_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

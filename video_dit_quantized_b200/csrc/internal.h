@@ -49,6 +49,10 @@ cudaError_t launch_quant_blocks_2d(const void* x, int R, int K, int8_t* codes, f
 cudaError_t launch_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias,
                                void* y, int y_f32, int M, int N, int K, uint32_t* status, long long timeout_cycles,
                                int dbg_flags, cudaStream_t stream);
+cudaError_t launch_dequant_blocks_2d(const int8_t* codes, const float* scales, int R, int K, void* out,
+                                     cudaStream_t stream);
+cudaError_t launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_f32, int M, int N,
+                               int K, uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream);
 
 // Diagnostics.
 cudaError_t launch_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int BH, int H, int N, int d,

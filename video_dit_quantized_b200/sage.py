@@ -62,6 +62,10 @@ def _load() -> ctypes.CDLL:
         "sage_quantize_blocks_2d": (i32, [vp, i32, i32, vp, vp, vp]),
         "sage_linear_w8a8": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
         "sage_dbg_linear_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
+        "sage_dequant_blocks_2d": (i32, [vp, vp, i32, i32, vp, vp]),
+        "sage_linear_bf16": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
+        "sage_linear_w8a16_workspace_bytes": (sz, [i32, i32]),
+        "sage_linear_w8a16": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -292,6 +296,51 @@ def linear_w8a8(xq, sx, wq, sw, bias=None, y=None, out_dtype=None, status=None, 
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
     _check(LIB.sage_linear_w8a8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M, N, K,
                                 _ptr(status), _stream(stream)), "sage_linear_w8a8")
+    return y
+
+
+def dequant_blocks_2d(codes, scales, out=None, stream=None):
+    """int8 codes [R, K] + block scales -> bf16 [R, K] = bf16(scale * code)."""
+    import torch
+    R, K = codes.shape
+    if out is None:
+        out = torch.empty((R, K), dtype=torch.bfloat16, device=codes.device)
+    _check(LIB.sage_dequant_blocks_2d(_ptr(codes), _ptr(scales), R, K, _ptr(out), _stream(stream)),
+           "sage_dequant_blocks_2d")
+    return out
+
+
+def linear_bf16(x, w, bias=None, y=None, out_dtype=None, status=None, stream=None):
+    """Y = X W^T + bias for bf16 X [M, K] and W [N, K]; returns Y [M, N]."""
+    import torch
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
+    if status is None:
+        status = torch.zeros(64, dtype=torch.int32, device=x.device)
+    code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
+    _check(LIB.sage_linear_bf16(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), code, M, N, K, _ptr(status),
+                                _stream(stream)), "sage_linear_bf16")
+    return y
+
+
+def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, status=None, stream=None):
+    """W8A16 layer: bf16 X [M, K] against 128 x 128 block-quantized W (wq int8 [N, K], sw); returns Y [M, N]."""
+    import torch
+    M, K = x.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
+    if status is None:
+        status = torch.zeros(64, dtype=torch.int32, device=x.device)
+    nbytes = int(LIB.sage_linear_w8a16_workspace_bytes(N, K))
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
+    _check(LIB.sage_linear_w8a16(_ptr(x), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M, N, K, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)),
+           "sage_linear_w8a16")
     return y
 
 
