@@ -15,7 +15,9 @@ HBM.  Metric: attention TFLOPS = 4 * B * H * N^2 * d / step time.
 instead (one step = block-quantize the activations X [M, K] + the block-scaled
 INT8 GEMM against pre-quantized weights W [N, K], plus bias), at the
 Wan2.1-14B 720p projection shape 75600 x 5120 x 5120 by default; metric
-TOPS = 2 * M * N * K / step time.
+TOPS = 2 * M * N * K / step time.  `--linear-mode w8a16` times the W8A16
+fallback (dequantize the 8-bit weights + bf16 GEMM), `--linear-mode bf16` the
+plain bf16 layer.
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 device (independent attention calls; no data-path collective), so scaling is
@@ -74,6 +76,7 @@ def parse():
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--op", default="attention", choices=["attention", "linear"])
     ap.add_argument("--linear-workload", default="wan14b_720p_proj", choices=sorted(synth.LINEAR_WORKLOADS))
+    ap.add_argument("--linear-mode", default="w8a8", choices=["w8a8", "w8a16", "bf16"])
     return ap.parse_args()
 
 
@@ -442,6 +445,8 @@ def run_linear(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     nk = w.K // 128
     wq, sw = sage.quantize_blocks_2d(wt)                  # weights: quantized once, outside the step
+    lmode = args.linear_mode
+    ws16 = torch.empty(int(sage.LIB.sage_linear_w8a16_workspace_bytes(w.N, w.K)), dtype=torch.uint8, device=dev)
     xq = torch.empty((w.M, w.K), dtype=torch.int8, device=dev)
     sx = torch.empty(((w.M + 127) // 128, nk), dtype=torch.float32, device=dev)
     y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
@@ -451,17 +456,27 @@ def run_linear(args, rank, world, local_rank):
     P = sage._ptr
 
     def step(ev=None):
+        """w8a8: quantize X | GEMM; w8a16: dequantize W | bf16 GEMM; bf16: - | bf16 GEMM."""
         if ev:
             ev[0].record(stream)
-        rc = sage.LIB.sage_quantize_blocks_2d(P(x), w.M, w.K, P(xq), P(sx), sp)
+        if lmode == "w8a8":
+            rc = sage.LIB.sage_quantize_blocks_2d(P(x), w.M, w.K, P(xq), P(sx), sp)
+        elif lmode == "w8a16":
+            rc = sage.LIB.sage_dequant_blocks_2d(P(wq), P(sw), w.N, w.K, P(ws16), sp)
+        else:
+            rc = 0
         if rc:
-            raise sage.SageError(rc, "sage_quantize_blocks_2d")
+            raise sage.SageError(rc, "quantize / dequantize")
         if ev:
             ev[1].record(stream)
-        rc = sage.LIB.sage_linear_w8a8(P(xq), P(sx), P(wq), P(sw), P(bias), P(y), sage.DTYPE_BF16, w.M, w.N, w.K,
-                                       P(status), sp)
+        if lmode == "w8a8":
+            rc = sage.LIB.sage_linear_w8a8(P(xq), P(sx), P(wq), P(sw), P(bias), P(y), sage.DTYPE_BF16, w.M, w.N, w.K,
+                                           P(status), sp)
+        else:
+            rc = sage.LIB.sage_linear_bf16(P(x), P(ws16 if lmode == "w8a16" else wt), P(bias), P(y), sage.DTYPE_BF16,
+                                           w.M, w.N, w.K, P(status), sp)
         if rc:
-            raise sage.SageError(rc, "sage_linear_w8a8")
+            raise sage.SageError(rc, "linear")
         if ev:
             ev[2].record(stream)
 
@@ -496,8 +511,13 @@ def run_linear(args, rank, world, local_rank):
 
     def e2e_step():
         x.copy_(x_h, non_blocking=True)
-        sage.quantize_blocks_2d(x, xq, sx, stream=stream)
-        sage.linear_w8a8(xq, sx, wq, sw, bias, y=y, status=status, stream=stream)
+        if lmode == "w8a8":
+            sage.quantize_blocks_2d(x, xq, sx, stream=stream)
+            sage.linear_w8a8(xq, sx, wq, sw, bias, y=y, status=status, stream=stream)
+        elif lmode == "w8a16":
+            sage.linear_w8a16(x, wq, sw, bias, y=y, workspace=ws16, status=status, stream=stream)
+        else:
+            sage.linear_bf16(x, wt, bias, y=y, status=status, stream=stream)
         y_h.copy_(y, non_blocking=True)
 
     e2e_step()
@@ -513,35 +533,39 @@ def run_linear(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), world, dev)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and lmode == "w8a8":
         cpu = cpu_baseline_linear(w, 1024)
         cpu.pop("seconds", None)
     if rank != 0:
         return
     ms_step = total_ms / args.steps
     peaks, src = load_peaks()
-    peak = 2.0 * float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    ratio = 2.0 if lmode == "w8a8" else 1.0
+    peak = ratio * float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     gemm_avg = statistics.mean(gemm_ms)
     achieved = w.flops / (gemm_avg * 1e-3) / 1e12
     line = {
-        "op": "linear_w8a8",
-        "metric": "W8A8 linear TOPS per call (2*M*N*K)",
+        "op": f"linear_{lmode}",
+        "metric": f"{lmode.upper()} linear TOPS per call (2*M*N*K)",
         "value": world * w.flops / (ms_step * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8 (int32 block sums, fp32 accumulate)", "data": "synthetic",
+        "vs_baseline": None,
+        "dtype": "int8 (int32 block sums, fp32 accumulate)" if lmode == "w8a8" else "bf16 (fp32 accumulate)",
+        "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "global_batch": world,
                    "parallelism": f"independent calls x{world}",
                    "l2": "X (774 MB bf16) larger than L2; no flush"},
-        "kernels_ms": {"quantize_median": statistics.median(quant_ms), "gemm_median": statistics.median(gemm_ms),
+        "kernels_ms": {("quantize_median" if lmode == "w8a8" else "dequantize_median"): statistics.median(quant_ms),
+                       "gemm_median": statistics.median(gemm_ms),
                        "gemm_min": min(gemm_ms), "gemm_max": max(gemm_ms)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": NCU_TRAFFIC_BYTES_LINEAR.get((w.name, "w8a8")),
-                     "peak_basis": f"2x bf16_tflops_sustained ({src})",
-                     "frac_of_datasheet_4500": achieved / 4500.0},
+                     "traffic": NCU_TRAFFIC_BYTES_LINEAR.get((w.name, lmode)),
+                     "peak_basis": f"{'2x ' if ratio == 2 else ''}bf16_tflops_sustained ({src})",
+                     "frac_of_datasheet": achieved / (4500.0 if ratio == 2 else 2250.0)},
         "cpu_baseline": cpu,
         "e2e": {"value": world * w.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if lmode == "bf16" else 2) * args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
