@@ -55,17 +55,19 @@ NCU_TRAFFIC_BYTES = {
     ("wan14b_720p", 40, "int8_fp8"): 1.653e9,
     ("wan14b_720p", 40, "bf16"): 3.002e9,
 }
-# W8A8 GEMM DRAM bytes per launch (ncu capture of the same kernel, summarised in
-# profiles/linear_w8a8_wan14b_720p.md).  Absent keys report null.
+# Linear GEMM DRAM bytes per launch (ncu captures of the same kernels, summarised in
+# profiles/linear_{w8a8,bf16}_wan14b_720p.md), keyed by (workload, linear mode).
+# Absent keys report null.
 NCU_TRAFFIC_BYTES_LINEAR = {
-    ("wan14b_720p_proj", "w8a8"): 1.160e9,
+    ("wan14b_720p_proj", "w8a16"): 3.477e9,
 }
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 10 for attention, 400 for --op linear)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
@@ -573,6 +575,9 @@ def run_linear(args, rank, world, local_rank):
 
 def main():
     args = parse()
+    if args.steps is None:
+        # a linear step is ~2.5 ms: 400 steps keep the timed region (and its clock samples) near a second
+        args.steps = 400 if args.op == "linear" else 10
     args.e2e_steps = max(1, args.e2e_steps)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -711,7 +711,7 @@ cudaError_t launch_linear_bf16(const void* x, const void* w, const void* bias, v
   prm.n_tiles_m = (M + bf16g::BM - 1) / bf16g::BM;
   prm.n_tiles_n = (N + bf16g::BN - 1) / bf16g::BN;
   prm.n_tiles = prm.n_tiles_m * prm.n_tiles_n;
-  prm.group_m = (size_t)N * K * 2 > (64u << 20) ? 16 : 1;   // W beyond half of L2: grouped order
+  prm.group_m = 16;                             // grouped order (see tile_coords)
   prm.y_f32 = y_f32;
   prm.timeout = timeout_cycles;
   prm.dbg_flags = dbg_flags;
