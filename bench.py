@@ -59,6 +59,7 @@ NCU_TRAFFIC_BYTES = {
 # profiles/linear_{w8a8,bf16}_wan14b_720p.md), keyed by (workload, linear mode).
 # Absent keys report null.
 NCU_TRAFFIC_BYTES_LINEAR = {
+    ("wan14b_720p_proj", "w8a8"): 1.152e9,
     ("wan14b_720p_proj", "w8a16"): 3.477e9,
 }
 

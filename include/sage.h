@@ -22,6 +22,11 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Calls are asynchronous on that stream; no call synchronises except
  *    sage_status() and sage_attn_fwd_host().
+ *  - The device calls allocate nothing and never synchronise, so after one
+ *    eager call per device (which sets kernel attributes) they can be
+ *    captured into a CUDA graph and replayed; sage_status(),
+ *    sage_attn_fwd_host() and the first call of sage_quantize_qk_noalloc on
+ *    a device cannot.
  *  - Every function returns SAGE_OK (0) or a negative SAGE_E* code; none
  *    aborts or throws.  Argument errors are detected on the host before any
  *    launch.  Device-side failures (a bounded wait that ran out) are recorded
