@@ -296,6 +296,30 @@ int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const vo
                       int M, int N, int K, void* workspace, size_t workspace_bytes, void* status, void* stream);
 
 /*
+ * Layout permutations around the DeepSpeed-Ulysses all-to-all (TMAP write-up,
+ * "Optimising multi-GPU parallelism": the sequence is split over P GPUs, an
+ * all-to-all gives each GPU the whole sequence for H/P heads, attention runs
+ * head-parallel, a second all-to-all returns O to the sequence slices).  The
+ * collectives are the caller's (NCCL); these calls move rows of d bf16
+ * values, Hl = H / P, N = P * Nl:
+ *   SAGE_ULYSSES_SEND_QKV  src [B, Nl, H, d]      -> dst [P][B, Hl, Nl, d]
+ *   SAGE_ULYSSES_RECV_QKV  src [P][B, Hl, Nl, d]  -> dst [B, Hl, N, d]
+ *   SAGE_ULYSSES_SEND_O    src [B, Hl, N, d]      -> dst [P][B, Hl, Nl, d]
+ *   SAGE_ULYSSES_RECV_O    src [P][B, Hl, Nl, d]  -> dst [B, Nl, H, d]
+ * The [P] side has chunk_rows rows (of d values) between consecutive chunks
+ * (0: dense, B*Hl*Nl) and starts base_rows rows into its buffer, so several
+ * tensors can share one all-to-all buffer.  H % P == 0, d in {64, 128},
+ * B, Nl, P >= 1; pointers 16-byte aligned, src and dst disjoint.
+ * Asynchronous on `stream`.
+ */
+#define SAGE_ULYSSES_SEND_QKV 0
+#define SAGE_ULYSSES_RECV_QKV 1
+#define SAGE_ULYSSES_SEND_O 2
+#define SAGE_ULYSSES_RECV_O 3
+int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
+                         long long chunk_rows, long long base_rows, void* stream);
+
+/*
  * Reads and clears the device status word at the start of `workspace`
  * (synchronises `stream`).  Returns SAGE_OK, SAGE_ETIMEOUT if a bounded
  * device-side wait ran out since the last call, or SAGE_ELAUNCH if the stream

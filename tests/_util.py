@@ -59,3 +59,29 @@ def emul_and_exact(q, k, v, rows):
     o2, _ = oracle.attn_emul(pre, rows)
     o1 = oracle.attn_exact(q, k, v, rows)
     return pre, o2, o1
+
+
+def ulysses_ref_permute(src, dst, B, Nl, H, d, P, op):
+    """The four Ulysses layout moves written with torch reshapes / permutes (dense [P] side)."""
+    Hl = H // P
+    if op == 0:      # [B, Nl, H, d] -> [P, B, Hl, Nl, d]
+        dst.copy_(src.reshape(B, Nl, P, Hl, d).permute(2, 0, 3, 1, 4))
+    elif op == 1:    # [P, B, Hl, Nl, d] -> [B, Hl, P*Nl, d]
+        dst.copy_(src.reshape(P, B, Hl, Nl, d).permute(1, 2, 0, 3, 4).reshape(B, Hl, P * Nl, d))
+    elif op == 2:    # [B, Hl, P*Nl, d] -> [P, B, Hl, Nl, d]
+        dst.copy_(src.reshape(B, Hl, P, Nl, d).permute(2, 0, 1, 3, 4))
+    else:            # [P, B, Hl, Nl, d] -> [B, Nl, H, d]
+        dst.copy_(src.reshape(P, B, Hl, Nl, d).permute(1, 3, 0, 2, 4).reshape(B, Nl, H, d))
+    return dst
+
+
+def attention_per_head_ref(q, k, v, mode, o, workspace=None):
+    """softmax(q k^T / sqrt(d)) v per (b, h) in float64, rounded to o's dtype; [B, H, N, d]."""
+    import torch
+    B, H, N, d = q.shape
+    for b in range(B):
+        for h in range(H):
+            s = (q[b, h].double() @ k[b, h].double().T) / d ** 0.5
+            p = torch.softmax(s, dim=-1)
+            o[b, h] = (p @ v[b, h].double()).to(o.dtype)
+    return o

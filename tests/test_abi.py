@@ -14,6 +14,7 @@ EXPECTED = {
     "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
     "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
     "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
+    "sage_ulysses_permute",
 }
 
 
@@ -124,3 +125,14 @@ def test_bf16_and_w8a16_argument_validation_runs_on_the_host():
     assert lib.sage_linear_w8a16(fake, fake, fake, None, fake, 0, 64, 256, 192, fake, 10 ** 9, fake, s) == sage.EINVAL
     assert lib.sage_linear_w8a16(fake, fake, fake, None, fake, 0, 64, 256, 256, fake, 1000, fake, s) == sage.EWORKSPACE
     assert lib.sage_dequant_blocks_2d(fake, fake, 10, 100, fake, s) == sage.EINVAL
+
+
+def test_ulysses_permute_argument_validation_runs_on_the_host():
+    lib = sage.LIB
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21)
+    s = None
+    assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 128, 3, 0, 0, 0, s) == sage.EINVAL   # H % P
+    assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 96, 4, 0, 0, 0, s) == sage.EINVAL    # d
+    assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 128, 4, 7, 0, 0, s) == sage.EINVAL   # op
+    assert lib.sage_ulysses_permute(a, a, 1, 10, 40, 128, 4, 0, 0, 0, s) == sage.EINVAL   # in place
+    assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 128, 4, 0, 5, 0, s) == sage.EINVAL   # chunk < dense

@@ -65,3 +65,62 @@ def test_two_rank_gloo_max_and_independent_shards():
 def test_single_rank_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def _ulysses_rank(rank, world, port, result_q):
+    import os
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from _util import attention_per_head_ref, ulysses_ref_permute
+    from video_dit_quantized_b200 import sage
+    from video_dit_quantized_b200.ulysses import UlyssesAttention
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.Workload("uly", 1, 4, 96, 16, seed=3)
+        full = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) for a in synth.qkv_numpy(w)]
+        # [B, H, N, d] -> the sequence-parallel layout [B, N, H, d], this rank's token slice
+        Nl = w.N // world
+        mine = [t.permute(0, 2, 1, 3)[:, rank * Nl:(rank + 1) * Nl].contiguous() for t in full]
+
+        def a2a(out, inp):
+            return dist.all_to_all_single(out, inp, async_op=True)
+
+        ua = UlyssesAttention(w.B, Nl, w.H, w.d, world, mode=sage.MODE_BF16, device="cpu",
+                              permute=ulysses_ref_permute, attention=attention_per_head_ref, a2a=a2a)
+        ua.send("q", mine[0])          # q goes out before k and v exist, as a DiT block would issue it
+        ua.send("k", mine[1])
+        ua.send("v", mine[2])
+        out = ua.attend()
+        ref = attention_per_head_ref(*full, sage.MODE_BF16, torch.empty_like(full[0]))
+        want = ref.permute(0, 2, 1, 3)[:, rank * Nl:(rank + 1) * Nl]
+        result_q.put((rank, bool(torch.equal(out.view(torch.int16), want.contiguous().view(torch.int16)))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ulysses_exchange_two_gloo_ranks():
+    """Two CPU ranks run the Ulysses exchange around a per-head reference attention; each rank's
+    output slice equals single-process attention on the whole sequence, bit for bit."""
+    import multiprocessing as mp
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ulysses_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    results = dict(q.get(timeout=5) for _ in range(2))
+    assert results == {0: True, 1: True}

@@ -1,0 +1,105 @@
+"""Ulysses layout permutations on the GPU, and the whole exchange emulated on one GPU.
+
+The four row permutations of sage_ulysses_permute equal independent torch
+reshape/permute references bit for bit, dense and with a strided [P] side.
+With P ranks emulated on one device (the all-to-all done by slicing the P
+send buffers), the sequence-parallel path -- permute, exchange, quantized or
+BF16 attention on the local heads, permute back, exchange, permute -- gives
+the same bits as one attention call over all heads: attention has no
+cross-head term and the kernels treat every (b, h) alike.  The pattern is the
+DeepSpeed-Ulysses sequence parallelism of the TMAP write-up ("Optimising
+multi-GPU parallelism").
+"""
+import numpy as np
+import pytest
+
+import synth
+from _util import ulysses_ref_permute
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(a, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+@pytest.mark.parametrize("B,Nl,H,d,P", [(1, 96, 8, 128, 1), (1, 100, 8, 128, 2), (2, 37, 12, 64, 4),
+                                        (1, 1181, 40, 128, 8)])
+def test_permutes_match_reference(B, Nl, H, d, P, cuda_dev):
+    import torch
+    from video_dit_quantized_b200 import sage
+    g = torch.Generator(device="cpu").manual_seed(B * 1000 + Nl + H + P)
+    Hl, N = H // P, P * Nl
+    shapes_in = {0: (B, Nl, H, d), 1: (P, B, Hl, Nl, d), 2: (B, Hl, N, d), 3: (P, B, Hl, Nl, d)}
+    shapes_out = {0: (P, B, Hl, Nl, d), 1: (B, Hl, N, d), 2: (P, B, Hl, Nl, d), 3: (B, Nl, H, d)}
+    for op in range(4):
+        src = torch.randn(shapes_in[op], generator=g).to(torch.bfloat16).to(cuda_dev)
+        got = torch.empty(shapes_out[op], dtype=torch.bfloat16, device=cuda_dev)
+        sage.ulysses_permute(src, got, B, Nl, H, d, P, op)
+        want = ulysses_ref_permute(src, torch.empty_like(got), B, Nl, H, d, P, op)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), op
+    # strided [P] side: q, k, v interleaved as [P][3][B, Hl, Nl, d]
+    dense = B * Hl * Nl
+    x = torch.randn((3, B, Nl, H, d), generator=g).to(torch.bfloat16).to(cuda_dev)
+    buf = torch.zeros((P, 3, B, Hl, Nl, d), dtype=torch.bfloat16, device=cuda_dev)
+    for t in range(3):
+        sage.ulysses_permute(x[t], buf, B, Nl, H, d, P, 0, chunk_rows=3 * dense, base_rows=t * dense)
+    back = torch.empty_like(x)
+    for t in range(3):
+        want = ulysses_ref_permute(x[t], torch.empty((P, B, Hl, Nl, d), dtype=torch.bfloat16, device=cuda_dev),
+                                   B, Nl, H, d, P, 0)
+        assert torch.equal(buf[:, t].view(torch.int16), want.view(torch.int16))
+        sage.ulysses_permute(buf, back[t], B, Nl, H, d, P, 3, chunk_rows=3 * dense, base_rows=t * dense)
+    torch.cuda.synchronize()
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))       # op 3 inverts op 0
+
+
+@pytest.mark.parametrize("mode_name,P", [("int8_fp8", 4), ("bf16", 2), ("int8_fp8", 8)])
+def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
+    import torch
+    from video_dit_quantized_b200 import sage
+    from video_dit_quantized_b200.ulysses import UlyssesAttention
+    mode = {"int8_fp8": sage.MODE_INT8_FP8, "bf16": sage.MODE_BF16}[mode_name]
+    w = synth.Workload("uly", 1, 8, 8 * 160, 128, seed=5 + P, outlier_frac=0.01)
+    q, k, v = (_bf16(a, cuda_dev) for a in synth.qkv_numpy(w))            # [B, H, N, d]
+    ref = sage.attn_fwd(q, k, v, mode)
+    Nl = w.N // P
+    seq = [t.permute(0, 2, 1, 3).contiguous() for t in (q, k, v)]         # [B, N, H, d]
+
+    # P ranks on one device; the all-to-all is done by hand once every rank has sent
+    sent = {}
+
+    def make_a2a(rank):
+        def a2a(out, inp):
+            sent[(rank, id(out))] = (out, inp)
+            return None
+        return a2a
+
+    ranks = [UlyssesAttention(w.B, Nl, w.H, w.d, P, mode=mode, device=cuda_dev, a2a=make_a2a(r))
+             for r in range(P)]
+
+    def exchange():
+        # rank r receives chunk r of every rank's send buffer, in rank order
+        outs = {}
+        for (r, _), (out, inp) in sent.items():
+            outs.setdefault(r, []).append((out, inp))
+        for slot in range(len(outs[0])):
+            for r in range(P):
+                out_r = outs[r][slot][0]
+                for src in range(P):
+                    out_r[src].copy_(outs[src][slot][1][r])
+        sent.clear()
+
+    for r, ua in enumerate(ranks):
+        for t, x in zip("qkv", seq):
+            ua.send(t, x[:, r * Nl:(r + 1) * Nl])
+    exchange()
+    for ua in ranks:
+        ua.attend_local()
+    exchange()
+    outs = [ua.finish().clone() for ua in ranks]
+    torch.cuda.synchronize()
+    got = torch.cat(outs, dim=1).permute(0, 2, 1, 3)                      # back to [B, H, N, d]
+    assert torch.equal(got.contiguous().view(torch.int16), ref.view(torch.int16))

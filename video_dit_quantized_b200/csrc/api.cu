@@ -389,6 +389,21 @@ int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const vo
                                           static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0, st));
 }
 
+int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
+                         long long chunk_rows, long long base_rows, void* stream) {
+  if (B < 1 || Nl < 1 || H < 1 || P < 1 || H % P != 0 || (d != 64 && d != 128)) return SAGE_EINVAL;
+  if (op < SAGE_ULYSSES_SEND_QKV || op > SAGE_ULYSSES_RECV_O || chunk_rows < 0 || base_rows < 0) return SAGE_EINVAL;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst) || src == dst) return SAGE_EINVAL;
+  const long long rows = (long long)B * Nl * H;
+  const long long dense = (long long)B * (H / P) * Nl;
+  if (chunk_rows != 0 && chunk_rows < dense) return SAGE_EINVAL;
+  if (rows * (d / 8) >= (1LL << 40)) return SAGE_EINVAL;
+  const int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  return launch_status(launch_ulysses_permute(src, dst, B, Nl, H, d, P, op, chunk_rows, base_rows,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 int sage_status(void* workspace, void* stream) {
   if (!workspace) return SAGE_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

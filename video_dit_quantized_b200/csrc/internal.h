@@ -54,6 +54,10 @@ cudaError_t launch_dequant_blocks_2d(const int8_t* codes, const float* scales, i
 cudaError_t launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_f32, int M, int N,
                                int K, uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream);
 
+// Ulysses layout permutations (op 0..3, see ulysses.cu).
+cudaError_t launch_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
+                                   long long chunk_rows, long long base_rows, cudaStream_t stream);
+
 // Diagnostics.
 cudaError_t launch_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int BH, int H, int N, int d,
                                 const int* tile_list, int n, int32_t* out, cudaStream_t stream);

@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
         "sage_linear_bf16": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
         "sage_linear_w8a16_workspace_bytes": (sz, [i32, i32]),
         "sage_linear_w8a16": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
+        "sage_ulysses_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, ll, ll, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -342,6 +343,17 @@ def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, s
                                  workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)),
            "sage_linear_w8a16")
     return y
+
+
+ULYSSES_SEND_QKV, ULYSSES_RECV_QKV, ULYSSES_SEND_O, ULYSSES_RECV_O = 0, 1, 2, 3
+
+
+def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, chunk_rows: int = 0,
+                    base_rows: int = 0, stream=None):
+    """Row permutation between the Ulysses layouts (see include/sage.h); dst is filled and returned."""
+    _check(LIB.sage_ulysses_permute(_ptr(src), _ptr(dst), B, Nl, H, d, P, op, int(chunk_rows), int(base_rows),
+                                    _stream(stream)), "sage_ulysses_permute")
+    return dst
 
 
 def status(workspace, stream=None) -> int:

@@ -1,0 +1,107 @@
+"""DeepSpeed-Ulysses sequence-parallel attention around the sage kernels.
+
+TMAP write-up, "Optimising multi-GPU parallelism": the sequence of a video
+DiT is split over P GPUs.  Before attention an all-to-all gives every GPU the
+whole sequence for H/P heads (attention is head-parallel, so the quantized
+kernels run unchanged on full sequences), and a second all-to-all returns
+the output to the sequence slices.  The all-to-all of q, k and v cost about
+2/3 of the attention time there, and the pages hide part of it by starting
+each exchange as soon as its tensor is computed, while the next projection
+still runs.  `UlyssesAttention.send` does exactly that: each of q, k, v is
+permuted into its send layout and its all-to-all is started at once
+(asynchronously, on the communicator's stream); `attend` waits for the three,
+runs the attention path on the local heads and brings O back.
+
+Per rank: inputs [B, Nl, H, d] (this rank's Nl = N / P tokens, all heads),
+output [B, Nl, H, d].  The permutations are the C ABI's
+`sage_ulysses_permute`; the collectives are torch.distributed's
+`all_to_all_single` (NCCL on GPUs).
+"""
+from __future__ import annotations
+
+from . import sage
+
+
+def _default_a2a(group):
+    import torch.distributed as dist
+
+    def a2a(out, inp):
+        return dist.all_to_all_single(out, inp, group=group, async_op=True)
+    return a2a
+
+
+class UlyssesAttention:
+    """One attention layer's Ulysses exchange for fixed shapes (buffers allocated once).
+
+    permute(src, dst, B, Nl, H, d, P, op) and attention(q, k, v, mode, o, workspace) default to the
+    CUDA kernels; a2a(out, inp) -> handle defaults to an asynchronous all_to_all_single on `group`.
+    """
+
+    def __init__(self, B: int, Nl: int, H: int, d: int, world: int, mode: int = sage.MODE_INT8_FP8,
+                 device=None, group=None, permute=None, attention=None, a2a=None):
+        import torch
+        if H % world:
+            raise ValueError(f"H={H} is not divisible by the {world} ranks")
+        self.B, self.Nl, self.H, self.d, self.P, self.mode = B, Nl, H, d, world, mode
+        self.Hl, self.N = H // world, world * Nl
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        bf = torch.bfloat16
+        chunk = (world, B, self.Hl, Nl, d)
+        self.send_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"}
+        self.recv_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"}
+        self.local = {t: torch.empty((B, self.Hl, self.N, d), dtype=bf, device=dev) for t in "qkv"}
+        self.o_local = torch.empty((B, self.Hl, self.N, d), dtype=bf, device=dev)
+        self.o_send = torch.empty(chunk, dtype=bf, device=dev)
+        self.o_recv = torch.empty(chunk, dtype=bf, device=dev)
+        self.out = torch.empty((B, Nl, H, d), dtype=bf, device=dev)
+        self.workspace = None
+        if attention is None and dev.type == "cuda":
+            self.workspace = sage.alloc_workspace(B, self.Hl, self.N, d, mode, dev)
+        self._permute = permute or (lambda src, dst, *g: sage.ulysses_permute(src, dst, *g))
+        self._attention = attention or (lambda q, k, v, m, o, ws: sage.attn_fwd(q, k, v, m, o=o, workspace=ws))
+        self._a2a = a2a or _default_a2a(group)
+        self._pending = {}
+
+    def _geom(self, op):
+        return (self.B, self.Nl, self.H, self.d, self.P, op)
+
+    def send(self, which: str, x):
+        """Start the exchange of q, k or v ([B, Nl, H, d] bf16): permute, then an async all-to-all."""
+        if which not in "qkv" or len(which) != 1:
+            raise ValueError("which must be 'q', 'k' or 'v'")
+        if tuple(x.shape) != (self.B, self.Nl, self.H, self.d):
+            raise ValueError(f"{which} must be [B, Nl, H, d] = {(self.B, self.Nl, self.H, self.d)}")
+        self._permute(x.contiguous(), self.send_buf[which], *self._geom(sage.ULYSSES_SEND_QKV))
+        self._pending[which] = self._a2a(self.recv_buf[which], self.send_buf[which])
+
+    def attend_local(self):
+        """Wait for q, k, v, run attention on the local heads and start O's way back."""
+        missing = [t for t in "qkv" if t not in self._pending]
+        if missing:
+            raise RuntimeError(f"send() was not called for {missing}")
+        for t in "qkv":
+            h = self._pending.pop(t)
+            if h is not None:
+                h.wait()
+            self._permute(self.recv_buf[t], self.local[t], *self._geom(sage.ULYSSES_RECV_QKV))
+        self._attention(self.local["q"], self.local["k"], self.local["v"], self.mode, self.o_local, self.workspace)
+        self._permute(self.o_local, self.o_send, *self._geom(sage.ULYSSES_SEND_O))
+        self._pending["o"] = self._a2a(self.o_recv, self.o_send)
+
+    def finish(self):
+        """Wait for O and return it for this rank's tokens, [B, Nl, H, d]."""
+        h = self._pending.pop("o")
+        if h is not None:
+            h.wait()
+        self._permute(self.o_recv, self.out, *self._geom(sage.ULYSSES_RECV_O))
+        return self.out
+
+    def attend(self):
+        """attend_local() then finish(): O [B, Nl, H, d] for this rank's tokens."""
+        self.attend_local()
+        return self.finish()
+
+    def __call__(self, q, k, v):
+        for t, x in zip("qkv", (q, k, v)):
+            self.send(t, x)
+        return self.attend()
