@@ -339,7 +339,7 @@ def run_ours(args, rank, world, local_rank):
     # copies its output out, overlapping the copies of one chunk with the
     # attention of another; every step moves all of Q, K, V in and all of O out.
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    chunk = (w.B * w.H + 7) // 8
+    chunk = sage.host_chunk_heads(w.B, w.H, w.N, w.d)
     ws_e2e = sage.alloc_workspace(1, chunk, w.N, w.d, mode, dev)
     staging = tuple(torch.empty_like(q) for _ in range(4))
     h2d = 3 * q.numel() * q.element_size()
@@ -400,7 +400,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * (4 if quant else 1),
-        "e2e_api": "sage_attn_fwd_host (pinned host Q/K/V in, O out, pipelined over 8 head chunks)",
+        "e2e_api": f"sage_attn_fwd_host (pinned host Q/K/V in, O out, pipelined over chunks of {chunk} heads)",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

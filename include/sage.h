@@ -174,7 +174,7 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
 
 /*
  * The same call from host memory, pipelined: the B*H heads are processed in
- * chunks of `chunk_heads` (0: B*H/8 rounded up); the host-to-device copy of
+ * chunks of `chunk_heads` (0: sage_host_chunk_heads()); the host-to-device copy of
  * chunk i+1 and the device-to-host copy of chunk i-1 overlap the attention of
  * chunk i.  Heads are independent (every statistic of the scheme is per head),
  * so the result is bit-for-bit that of sage_attn_fwd on the whole tensor.
@@ -191,6 +191,15 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H,
                        int N, int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
                        void* workspace, size_t workspace_bytes, int chunk_heads, void* stream);
+
+/*
+ * The default chunk of sage_attn_fwd_host: the fewest heads whose attention
+ * launch fills four waves of the current device's SMs (148 if no device is
+ * usable), at most B*H; 2 heads at the Wan2.1-14B 720p shape.  Small chunks
+ * leave less of the first upload and the last download uncovered.  0 on a
+ * bad shape.
+ */
+int sage_host_chunk_heads(int B, int H, int N, int d);
 
 /*
  * Per-layer mode table for selective quantization ("keeping video quality":

@@ -14,7 +14,7 @@ EXPECTED = {
     "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
     "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
     "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
-    "sage_ulysses_permute",
+    "sage_ulysses_permute", "sage_host_chunk_heads",
 }
 
 
@@ -136,3 +136,11 @@ def test_ulysses_permute_argument_validation_runs_on_the_host():
     assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 128, 4, 7, 0, 0, s) == sage.EINVAL   # op
     assert lib.sage_ulysses_permute(a, a, 1, 10, 40, 128, 4, 0, 0, 0, s) == sage.EINVAL   # in place
     assert lib.sage_ulysses_permute(a, b, 1, 10, 40, 128, 4, 0, 5, 0, s) == sage.EINVAL   # chunk < dense
+
+
+def test_host_chunk_rule():
+    # one CTA per 256 query rows of a head; four waves of 148 SMs
+    assert sage.host_chunk_heads(1, 40, 75600, 128) == 2          # 296 CTAs per head
+    assert sage.host_chunk_heads(1, 30, 17776, 64) == 9           # 70 CTAs per head
+    assert sage.host_chunk_heads(1, 2, 1024, 128) == 2            # capped at B*H
+    assert sage.host_chunk_heads(1, 2, 1024, 96) == 0             # bad shape

@@ -211,6 +211,23 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
                                         kDefaultTimeoutCycles, 0, st, qtok));
 }
 
+int sage_host_chunk_heads(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d) != SAGE_OK) return 0;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  // the smallest chunk whose attention launch (one CTA per 256 query rows of a head) fills 4 waves
+  const long long ctas_per_head = (N + 255) / 256;
+  long long chunk = (4LL * sms + ctas_per_head - 1) / ctas_per_head;
+  const long long BH = (long long)B * H;
+  if (chunk < 1) chunk = 1;
+  if (chunk > BH) chunk = BH;
+  return (int)chunk;
+}
+
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H, int N,
                        int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev, void* workspace,
                        size_t workspace_bytes, int chunk_heads, void* stream) {
@@ -221,7 +238,7 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAGE_EINVAL;
   const int BH = B * H;
-  if (chunk_heads <= 0) chunk_heads = (BH + 7) / 8;
+  if (chunk_heads <= 0) chunk_heads = sage_host_chunk_heads(B, H, N, d);
   if (chunk_heads > BH) chunk_heads = BH;
   const int n_chunks = (BH + chunk_heads - 1) / chunk_heads;
   if (workspace_bytes < sage_workspace_bytes(1, chunk_heads, N, d, mode)) return SAGE_EWORKSPACE;

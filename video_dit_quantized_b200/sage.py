@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "sage_linear_w8a16_workspace_bytes": (sz, [i32, i32]),
         "sage_linear_w8a16": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
         "sage_ulysses_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, ll, ll, vp]),
+        "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -210,7 +211,7 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, c
     import torch
     B, H, N, d = _bhnd(q_h, "q_h")
     BH = B * H
-    chunk = chunk_heads if chunk_heads > 0 else (BH + 7) // 8
+    chunk = chunk_heads if chunk_heads > 0 else host_chunk_heads(B, H, N, d)
     chunk = min(chunk, BH)
     if staging is None:
         staging = tuple(torch.empty(q_h.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
@@ -346,6 +347,11 @@ def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, s
 
 
 ULYSSES_SEND_QKV, ULYSSES_RECV_QKV, ULYSSES_SEND_O, ULYSSES_RECV_O = 0, 1, 2, 3
+
+
+def host_chunk_heads(B: int, H: int, N: int, d: int) -> int:
+    """Default head chunk of attn_fwd_host (see sage_host_chunk_heads)."""
+    return int(LIB.sage_host_chunk_heads(B, H, N, d))
 
 
 def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, chunk_rows: int = 0,
