@@ -63,3 +63,43 @@ def test_calibration_selects_the_outlier_layers(cuda_dev):
     np.testing.assert_allclose(err.mean(1), np.mean(oracle_err, 1), rtol=0.35)
     modes = sage.layer_schedule(4, picked)
     assert modes == [sage.MODE_INT8_FP8, sage.MODE_BF16, sage.MODE_INT8_FP8, sage.MODE_BF16]
+
+
+def test_linear_layer_selection_matches_the_oracle(cuda_dev):
+    """Selective W8A8 -> W8A16 for linear layers: on a synthetic stack where two layers carry strong
+    activation outlier channels (per-block X scales inflated by 100x outliers), the layers whose
+    W8A8-vs-W8A16 error exceeds the threshold are the ones the oracle's errors select."""
+    import torch
+    from video_dit_quantized_b200 import sage
+    L, iters = 6, 2
+    heavy = {2, 5}
+    layers, oracle_err = [], []
+    for l in range(L):
+        row, orow = [], []
+        for it in range(iters):
+            lw = synth.LinearWorkload("cal", 256, 256, 512, seed=100 * l + it,
+                                      outlier_frac=0.02, outlier_scale=100.0 if l in heavy else 3.0)
+            x, wt, b = synth.linear_numpy(lw)
+            dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(cuda_dev)
+            wq, sw = sage.quantize_blocks_2d(dev(wt))
+            row.append((dev(x), wq, sw, dev(b)))
+            # oracle: W8A8 (fp32, then bf16) against W8A16 (exact product of the dequantized weights)
+            xq_o, sx_o = oracle.quant_blocks_2d(x)
+            wq_o, sw_o = oracle.quant_blocks_2d(wt)
+            _, y8 = oracle.linear_w8a8(xq_o, sx_o, wq_o, sw_o, b)
+            y16 = oracle.linear_bf16(x, oracle.dequant_blocks_2d(wq_o, sw_o), b)
+            y16 = torch.from_numpy(y16).to(torch.bfloat16).double().numpy()    # both outputs are bf16
+            a = synth.bf16_bits_to_f32(y8).astype(np.float64)
+            orow.append(float(np.linalg.norm(a - y16) / np.linalg.norm(y16)))
+        layers.append(row)
+        oracle_err.append(orow)
+    err = sage.linear_layer_errors(layers)
+    # the same errors: the W8A8 outputs are bit-exact; the W8A16 ones differ only by fp32 summation order
+    np.testing.assert_allclose(err, oracle_err, rtol=0.02)
+    light = [np.mean(oracle_err[l]) for l in range(L) if l not in heavy]
+    strong = [np.mean(oracle_err[l]) for l in heavy]
+    assert min(strong) > 2 * max(light)                         # the synthetic stack separates the two kinds
+    thr = float(np.sqrt(max(light) * min(strong)))
+    picked = sage.select_full_precision_layers(err, thr)
+    assert picked == sorted(heavy)
+    assert picked == [l for l in range(L) if np.mean(oracle_err[l]) > thr]

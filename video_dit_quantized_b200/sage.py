@@ -254,6 +254,28 @@ def layer_errors(layers, stream=None):
     return out
 
 
+def linear_layer_errors(layers, stream=None):
+    """Relative L2 error of the W8A8 output against the W8A16 output, per linear layer and iteration.
+
+    The FFN section's selective quantization for linear layers: the weights stay 8-bit in both modes,
+    so the error measured here is what quantizing the activations costs; the layers whose error stays
+    large run W8A16 (select_full_precision_layers on this table).
+    layers: [num_layers][num_iters] of (x bf16 [M, K], wq int8 [N, K], sw fp32, bias bf16 [N] or None).
+    """
+    out = []
+    for per_layer in layers:
+        row = []
+        for (x, wq, sw, bias) in per_layer:
+            xq, sx = quantize_blocks_2d(x, stream=stream)
+            y8 = linear_w8a8(xq, sx, wq, sw, bias, stream=stream)
+            y16 = linear_w8a16(x, wq, sw, bias, stream=stream)
+            M, N = y8.shape
+            st = error_stats(y8.view(1, 1, M, N), y16.view(1, 1, M, N), stream=stream).sum(dim=0).cpu()
+            row.append(float((st[0] / st[1]).sqrt()))
+        out.append(row)
+    return out
+
+
 def select_full_precision_layers(layer_err, threshold: float) -> list[int]:
     """Layers whose mean error over iterations exceeds threshold; layer_err is [layers][iterations]."""
     import numpy as np
