@@ -365,6 +365,8 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_rows)
         cpu.pop("seconds", None)
+    # the tensor-core rate the kernel is bounded by, measured per SM per clock on this GPU (MMA-only probe)
+    probe = sage.dbg_mma_peak(sage.MMA_I8 if quant else sage.MMA_BF16, 256, iters=2000)
 
     if rank != 0:
         return
@@ -400,6 +402,11 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * (4 if quant else 1),
+        "mma_probe": {"kind": "i8" if quant else "bf16", "mac_per_clk_per_sm": probe["mac_per_clk_per_sm"],
+                      "peak_at_median_sm_clock_tflops": (2 * probe["mac_per_clk_per_sm"] * probe["sms"] *
+                                                         (clocks["sm_mhz"] or 0) * 1e6 / 1e12),
+                      "frac_of_it": (achieved / (2 * probe["mac_per_clk_per_sm"] * probe["sms"] *
+                                                 clocks["sm_mhz"] * 1e6 / 1e12)) if clocks["sm_mhz"] else None},
         "e2e_api": f"sage_attn_fwd_host (pinned host Q/K/V in, O out, pipelined over chunks of {chunk} heads)",
         "clocks": clocks,
     }

@@ -392,6 +392,21 @@ int sage_dbg_linear_forced_timeout(const int8_t* xq, const float* sx, const int8
                                    const void* bias, void* y, int y_dtype, int M, int N, int K, void* status,
                                    long long timeout_cycles, void* stream);
 
+/*
+ * Tensor-core throughput probe: one CTA per SM (grid = the device's SM
+ * count) issues `iters` x 4 back-to-back tcgen05.mma of M=128, N = n (128 or
+ * 256) and 32 bytes of K from shared-memory operands into tensor memory, and
+ * writes each CTA's elapsed SM clocks to cycles (device int64 [grid]).
+ * kind: SAGE_MMA_BF16 (K = 16 bf16), SAGE_MMA_E4M3 (K = 32), SAGE_MMA_I8
+ * (K = 32).  MACs per SM per clock = iters * 4 * 128 * n * K / cycles.
+ * status as for sage_attn_quantized.  Not part of the attention or linear
+ * paths; it measures the rate they are bounded by, at any SM clock.
+ */
+#define SAGE_MMA_BF16 0
+#define SAGE_MMA_E4M3 1
+#define SAGE_MMA_I8 2
+int sage_dbg_mma_peak(int kind, int n, int iters, long long* cycles, int grid, void* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -81,3 +81,13 @@ def test_qk_bf16_tile(d, cuda_dev):
     Q, K = q.double().numpy(), k.double().numpy()
     want = Q @ K.T
     assert np.all(np.abs(got - want) <= 1e-5 * (np.abs(Q) @ np.abs(K).T) + 1e-30)
+
+
+def test_mma_throughput_probe(cuda_dev):
+    """Dense tcgen05 rates per SM per clock: 8192 MACs for kind::i8 and kind::f8f6f4, 4096 for kind::f16
+    (twice the bf16 rate for 8-bit, as the datasheet's 4.5 vs 2.25 PFLOP/s), at N = 128 and 256."""
+    from video_dit_quantized_b200 import sage
+    for kind, want in ((sage.MMA_I8, 8192), (sage.MMA_E4M3, 8192), (sage.MMA_BF16, 4096)):
+        for n in (128, 256):
+            r = sage.dbg_mma_peak(kind, n, iters=2000)
+            assert 0.95 * want <= r["mac_per_clk_per_sm"] <= 1.01 * want, (kind, n, r)

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "prepass.cu", "attention.cu", "noalloc.cu", "calib.cu", "linear.cu", "ulysses.cu"]
+SOURCES = ["api.cu", "prepass.cu", "attention.cu", "noalloc.cu", "calib.cu", "linear.cu", "ulysses.cu", "diag.cu"]
 HEADERS = ["internal.h", "sm100.cuh"]
 LIB_PATH = os.path.join(HERE, "libsage.so")
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -421,6 +421,17 @@ int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int sage_dbg_mma_peak(int kind, int n, int iters, long long* cycles, int grid, void* status, void* stream) {
+  if (kind < SAGE_MMA_BF16 || kind > SAGE_MMA_I8 || (n != 128 && n != 256) || iters < 1 || grid < 1) return SAGE_EINVAL;
+  if (!cycles || !status || (reinterpret_cast<uintptr_t>(cycles) & 7u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return SAGE_EINVAL;
+  const int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  // SAGE_MMA_* follow the kind numbering of the kernels (f16, f8f6f4, i8)
+  return launch_status(launch_mma_peak(kind, n, iters, cycles, static_cast<uint32_t*>(status), grid,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int sage_status(void* workspace, void* stream) {
   if (!workspace) return SAGE_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

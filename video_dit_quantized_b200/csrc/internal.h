@@ -58,6 +58,10 @@ cudaError_t launch_linear_bf16(const void* x, const void* w, const void* bias, v
 cudaError_t launch_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
                                    long long chunk_rows, long long base_rows, cudaStream_t stream);
 
+// Tensor-core throughput probe (kind: kKindF16 / kKindF8F6F4 / kKindI8 of sm100.cuh; n 128 or 256).
+cudaError_t launch_mma_peak(int kind, int n, int iters, long long* cycles, uint32_t* status, int grid,
+                            cudaStream_t stream);
+
 // Diagnostics.
 cudaError_t launch_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int BH, int H, int N, int d,
                                 const int* tile_list, int n, int32_t* out, cudaStream_t stream);

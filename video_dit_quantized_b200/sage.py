@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "sage_linear_w8a16": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
         "sage_ulysses_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, ll, ll, vp]),
         "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
+        "sage_dbg_mma_peak": (i32, [i32, i32, i32, vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -443,6 +444,25 @@ def dbg_linear_forced_timeout(xq, sx, wq, sw, status, timeout_cycles: int, bias=
                                               N, K, _ptr(status), int(timeout_cycles), _stream(stream)),
            "sage_dbg_linear_forced_timeout")
     return y
+
+
+MMA_BF16, MMA_E4M3, MMA_I8 = 0, 1, 2
+
+
+def dbg_mma_peak(kind: int, n: int = 256, iters: int = 4000, stream=None) -> dict:
+    """Tensor-core probe: MACs per SM per clock of back-to-back tcgen05.mma (slowest SM)."""
+    import torch
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device="cuda")
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    _check(LIB.sage_dbg_mma_peak(int(kind), int(n), int(iters), _ptr(cycles), sms, _ptr(status), _stream(stream)),
+           "sage_dbg_mma_peak")
+    torch.cuda.synchronize()
+    if int(status[0].item()) != 0:
+        raise SageError(ETIMEOUT, "sage_dbg_mma_peak")
+    k = 16 if kind == MMA_BF16 else 32
+    slowest = int(cycles.max().item())
+    return {"mac_per_clk_per_sm": iters * 4 * 128 * n * k / slowest, "cycles": slowest, "sms": sms}
 
 
 def dbg_attn_forced_timeout(pre: dict, N: int, status, timeout_cycles: int, o=None, stream=None):
