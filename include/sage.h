@@ -393,6 +393,14 @@ int sage_dbg_linear_forced_timeout(const int8_t* xq, const float* sx, const int8
                                    long long timeout_cycles, void* stream);
 
 /*
+ * The same test hook for sage_linear_bf16: its MMA thread first waits on a
+ * barrier no one completes, with a limit of `timeout_cycles` SM clocks, so
+ * the kernel records SAGE_ETIMEOUT in `status` and returns without hanging.
+ */
+int sage_dbg_linear_bf16_forced_timeout(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M,
+                                        int N, int K, void* status, long long timeout_cycles, void* stream);
+
+/*
  * Tensor-core throughput probe: one CTA per SM (grid = the device's SM
  * count) issues `iters` x 4 back-to-back tcgen05.mma of M=128, N = n (128 or
  * 256) and 32 bytes of K from shared-memory operands into tensor memory, and

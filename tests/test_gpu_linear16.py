@@ -126,3 +126,20 @@ def test_linear_bf16_full_size_sampled_rows(cuda_dev):
     got = y[torch.from_numpy(rows).long().to(cuda_dev)].cpu().numpy()
     got16 = torch.from_numpy(got).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     _check(got, got16, x, deq_o, b, rows, w.K)
+
+
+def test_linear_bf16_forced_timeout_reports_and_recovers(cuda_dev):
+    import torch
+    from video_dit_quantized_b200 import sage
+    w = synth.LINEAR_WORKLOADS["lin_tiny"]
+    x, wt, b = synth.linear_numpy(w)
+    xd, wd, bd = _bf16_dev(x, cuda_dev), _bf16_dev(wt, cuda_dev), _bf16_dev(b, cuda_dev)
+    st = torch.zeros(64, dtype=torch.int32, device=cuda_dev)
+    sage.dbg_linear_bf16_forced_timeout(xd, wd, st, timeout_cycles=2_000_000, bias=bd)
+    assert sage.status(st) == sage.ETIMEOUT
+    assert sage.status(st) == sage.OK
+    y = sage.linear_bf16(xd, wd, bd, out_dtype=torch.float32, status=st)     # the context is still usable
+    torch.cuda.synchronize()
+    assert sage.status(st) == sage.OK
+    _check(y.cpu().numpy(), y.to(torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16), x, wt, b,
+           np.arange(w.M), w.K)

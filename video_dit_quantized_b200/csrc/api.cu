@@ -386,6 +386,17 @@ int sage_linear_bf16(const void* x, const void* w, const void* bias, void* y, in
                                           static_cast<cudaStream_t>(stream)));
 }
 
+int sage_dbg_linear_bf16_forced_timeout(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M,
+                                        int N, int K, void* status, long long timeout_cycles, void* stream) {
+  if (timeout_cycles < 1) return SAGE_EINVAL;
+  int rc = check_linear_bf16(x, w, bias, y, y_dtype, M, N, K, status);
+  if (rc != SAGE_OK) return rc;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  return launch_status(launch_linear_bf16(x, w, bias, y, y_dtype == SAGE_DTYPE_F32, M, N, K,
+                                          static_cast<uint32_t*>(status), timeout_cycles, 1,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 size_t sage_linear_w8a16_workspace_bytes(int N, int K) {
   if (N < 1 || K < 1) return 0;
   return align_up((size_t)N * K * 2, 256);

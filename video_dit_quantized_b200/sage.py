@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "sage_ulysses_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, ll, ll, vp]),
         "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
         "sage_dbg_mma_peak": (i32, [i32, i32, i32, vp, i32, vp, vp]),
+        "sage_dbg_linear_bf16_forced_timeout": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -443,6 +444,19 @@ def dbg_linear_forced_timeout(xq, sx, wq, sw, status, timeout_cycles: int, bias=
     _check(LIB.sage_dbg_linear_forced_timeout(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M,
                                               N, K, _ptr(status), int(timeout_cycles), _stream(stream)),
            "sage_dbg_linear_forced_timeout")
+    return y
+
+
+def dbg_linear_bf16_forced_timeout(x, w, status, timeout_cycles: int, bias=None, y=None, stream=None):
+    import torch
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
+    _check(LIB.sage_dbg_linear_bf16_forced_timeout(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), code, M, N, K, _ptr(status),
+                                                   int(timeout_cycles), _stream(stream)),
+           "sage_dbg_linear_bf16_forced_timeout")
     return y
 
 
