@@ -68,7 +68,7 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 10 for attention, 400 for --op linear)")
+                    help="timed steps (default: 20 for attention, 400 for --op linear)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
@@ -328,6 +328,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = t_start.elapsed_time(t_end)
     prep_ms = [a.elapsed_time(b) for a, b, _ in evs]
     attn_ms = [b.elapsed_time(c) for _, b, c in evs]
+    step_ms = [a.elapsed_time(c) for a, _, c in evs]
     st = sage.status(ws)
     if st != sage.OK:
         raise sage.SageError(st, "timed region")
@@ -393,7 +394,10 @@ def run_ours(args, rank, world, local_rank):
                    "global_batch": world * w.B, "parallelism": f"independent calls x{world}",
                    "l2": "inputs (2.3 GB) larger than L2; no flush"},
         "kernels_ms": {"prepass_median": statistics.median(prep_ms), "attention_median": statistics.median(attn_ms),
-                       "attention_min": min(attn_ms), "attention_max": max(attn_ms)},
+                       "attention_p10": float(np.percentile(attn_ms, 10)),
+                       "attention_p90": float(np.percentile(attn_ms, 90)),
+                       "attention_min": min(attn_ms), "attention_max": max(attn_ms),
+                       "step_p10": float(np.percentile(step_ms, 10)), "step_p90": float(np.percentile(step_ms, 90))},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_basis": f"{'2x ' if ratio == 2 else ''}bf16_tflops_sustained ({src})",
@@ -585,7 +589,7 @@ def main():
     args = parse()
     if args.steps is None:
         # a linear step is ~2.5 ms: 400 steps keep the timed region (and its clock samples) near a second
-        args.steps = 400 if args.op == "linear" else 10
+        args.steps = 400 if args.op == "linear" else 20
     args.e2e_steps = max(1, args.e2e_steps)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
