@@ -11,6 +11,13 @@ HBM.  Metric: attention TFLOPS = 4 * B * H * N^2 * d / step time.
                   [--workload NAME] [--mode int8_fp8|bf16]
   python bench.py --op linear [--linear-workload NAME]
 
+`--op ulysses` times the sequence-parallel layer instead: each of N ranks holds
+N_seq / N tokens of Q, K, V for all heads; the Ulysses exchange (NCCL
+all-to-all) gives each the whole sequence for H / N heads, the INT8/FP8 path
+runs on them, and O goes back.  The total problem is fixed (strong scaling);
+value = the full layer's attention FLOPs / max-over-ranks time.  On one GPU
+the exchange is a single-rank NCCL all-to-all (a local copy).
+
 `--op linear` times the W8A8 linear layer with 128 x 128 block scales
 instead (one step = block-quantize the activations X [M, K] + the block-scaled
 INT8 GEMM against pre-quantized weights W [N, K], plus bias), at the
@@ -77,7 +84,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3, help="end-to-end steps (at least 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4096)
-    ap.add_argument("--op", default="attention", choices=["attention", "linear"])
+    ap.add_argument("--op", default="attention", choices=["attention", "linear", "ulysses"])
     ap.add_argument("--linear-workload", default="wan14b_720p_proj", choices=sorted(synth.LINEAR_WORKLOADS))
     ap.add_argument("--linear-mode", default="w8a8", choices=["w8a8", "w8a16", "bf16"])
     return ap.parse_args()
@@ -585,6 +592,63 @@ def run_linear(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ulysses(args, rank, world, local_rank):
+    """Sequence-parallel attention layer: Ulysses exchange around the INT8/FP8 path."""
+    import torch
+    import torch.distributed as dist
+    from video_dit_quantized_b200 import sage
+    from video_dit_quantized_b200.ulysses import UlyssesAttention
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(args)
+    if w.N % world or w.H % world:
+        raise SystemExit(f"N={w.N} and H={w.H} must be divisible by the {world} ranks")
+    Nl = w.N // world
+    mode = {"int8_fp8": sage.MODE_INT8_FP8, "bf16": sage.MODE_BF16, "int8_fp8_qtoken": sage.MODE_INT8_FP8_QTOKEN}[args.mode]
+    full = synth.qkv_torch(w)                                   # the same seeded layer on every rank
+    mine = [t.permute(0, 2, 1, 3)[:, rank * Nl:(rank + 1) * Nl].contiguous().to(dev) for t in full]
+    del full
+    ua = UlyssesAttention(w.B, Nl, w.H, w.d, world, mode=mode, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ua(*mine)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sage.status(ua.workspace) != sage.OK:
+        raise sage.SageError(sage.ETIMEOUT, "warm-up")
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    if sage.status(ua.workspace) != sage.OK:
+        raise sage.SageError(sage.ETIMEOUT, "timed region")
+    if rank != 0:
+        return
+    print(json.dumps({
+        "op": "ulysses_attention",
+        "metric": "attention TFLOPS per call (4*B*H*N^2*d), sequence-parallel layer",
+        "value": w.flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "int8/fp8e4m3 (fp32 accumulate)" if mode != sage.MODE_BF16 else "bf16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
+                   "parallelism": f"ulysses sp{world}", "tokens_per_rank": Nl, "heads_per_rank": w.H // world},
+        "gpu_launches": args.steps * (3 + 3 + 4 + 2),         # permutes, prepass + attention, O permutes
+        "clocks": clk.summary(),
+    }), flush=True)
+
+
 def main():
     args = parse()
     if args.steps is None:
@@ -597,21 +661,28 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
-    if world > 1:
+    if world > 1 or args.op == "ulysses":
         import datetime
 
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.op == "linear":
+        if args.op == "ulysses":
+            run_ulysses(args, rank, world, local_rank)
+        elif args.op == "linear":
             run_linear(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
+        if world > 1 or args.op == "ulysses":
             import torch.distributed as dist
             dist.destroy_process_group()
 

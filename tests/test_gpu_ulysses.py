@@ -103,3 +103,33 @@ def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
     torch.cuda.synchronize()
     got = torch.cat(outs, dim=1).permute(0, 2, 1, 3)                      # back to [B, H, N, d]
     assert torch.equal(got.contiguous().view(torch.int16), ref.view(torch.int16))
+
+
+def test_single_rank_nccl_exchange(cuda_dev):
+    """The default communicator path: a one-rank NCCL group, all_to_all_single as the exchange."""
+    import os
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    from video_dit_quantized_b200 import sage
+    from video_dit_quantized_b200.ulysses import UlyssesAttention
+    w = synth.Workload("uly1", 1, 4, 640, 128, seed=9, outlier_frac=0.01)
+    q, k, v = (_bf16(a, cuda_dev) for a in synth.qkv_numpy(w))
+    ref = sage.attn_fwd(q, k, v, sage.MODE_INT8_FP8)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    group_made = False
+    try:
+        if not dist.is_initialized():
+            dist.init_process_group("nccl", store=store, rank=0, world_size=1, device_id=cuda_dev)
+            group_made = True
+        ua = UlyssesAttention(w.B, w.N, w.H, w.d, 1, mode=sage.MODE_INT8_FP8, device=cuda_dev)
+        out = ua(*(t.permute(0, 2, 1, 3).contiguous() for t in (q, k, v)))
+        torch.cuda.synchronize()
+        assert torch.equal(out.permute(0, 2, 1, 3).contiguous().view(torch.int16), ref.view(torch.int16))
+    finally:
+        if group_made:
+            dist.destroy_process_group()
