@@ -265,7 +265,8 @@ int sage_select_full_precision_layers(const double* layer_err, int num_layers, i
  * aligned; sx, sw 4-byte aligned.  status: device memory whose first uint32
  * is the status word (the workspace of the attention calls serves);
  * sage_status() on it reports a bounded wait that ran out.  Asynchronous on
- * `stream`.
+ * `stream`.  Errors: SAGE_EINVAL (sizes, null or misaligned pointers, bad
+ * y_dtype), SAGE_EUNSUPPORTED / SAGE_ELAUNCH (device), all before any launch.
  */
 #define SAGE_LIN_BLK 128
 #define SAGE_DTYPE_BF16 0
@@ -295,7 +296,9 @@ int sage_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const 
  * multiple of 128; workspace: device memory of at least
  * sage_linear_w8a16_workspace_bytes(N, K) bytes, 16-byte aligned.
  *
- * status as for sage_linear_w8a8.  Asynchronous on `stream`.
+ * status as for sage_linear_w8a8.  Asynchronous on `stream`.  Errors:
+ * SAGE_EINVAL (sizes, pointers, y_dtype), SAGE_EWORKSPACE (workspace too
+ * small), SAGE_EUNSUPPORTED / SAGE_ELAUNCH (device).
  */
 int sage_dequant_blocks_2d(const int8_t* codes, const float* scales, int R, int K, void* out, void* stream);
 int sage_linear_bf16(const void* x, const void* w, const void* bias, void* y, int y_dtype, int M, int N, int K,
@@ -319,7 +322,8 @@ int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const vo
  * (0: dense, B*Hl*Nl) and starts base_rows rows into its buffer, so several
  * tensors can share one all-to-all buffer.  H % P == 0, d in {64, 128},
  * B, Nl, P >= 1; pointers 16-byte aligned, src and dst disjoint.
- * Asynchronous on `stream`.
+ * Asynchronous on `stream`.  Errors: SAGE_EINVAL (sizes, op, chunk_rows
+ * below the dense chunk, pointers), SAGE_EUNSUPPORTED / SAGE_ELAUNCH (device).
  */
 #define SAGE_ULYSSES_SEND_QKV 0
 #define SAGE_ULYSSES_RECV_QKV 1
