@@ -124,3 +124,40 @@ def test_ulysses_exchange_two_gloo_ranks():
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     results = dict(q.get(timeout=5) for _ in range(2))
     assert results == {0: True, 1: True}
+
+
+def test_ulysses_host_checks():
+    """UlyssesAttention refuses what the exchange cannot do, on the host (no GPU, no process group)."""
+    import torch
+
+    from _util import attention_per_head_ref, ulysses_ref_permute
+    from video_dit_quantized_b200 import sage
+    from video_dit_quantized_b200.ulysses import UlyssesAttention
+
+    with pytest.raises(ValueError):
+        UlyssesAttention(1, 8, 6, 16, 4, device="cpu", permute=ulysses_ref_permute,
+                         attention=attention_per_head_ref, a2a=lambda o, i: None)      # 6 heads over 4 ranks
+    sent = []
+
+    def a2a(out, inp):
+        sent.append(inp.shape)
+        out.copy_(inp)                                   # one rank: the exchange is a copy
+        return None
+
+    ua = UlyssesAttention(1, 8, 4, 16, 1, mode=sage.MODE_BF16, device="cpu", permute=ulysses_ref_permute,
+                          attention=attention_per_head_ref, a2a=a2a)
+    x = torch.randn(1, 8, 4, 16).to(torch.bfloat16)
+    with pytest.raises(ValueError):
+        ua.send("q", torch.randn(1, 8, 2, 16).to(torch.bfloat16))                    # wrong shape
+    with pytest.raises(ValueError):
+        ua.send("x", x)
+    ua.send("q", x)
+    with pytest.raises(RuntimeError):
+        ua.attend()                                                                  # k and v not sent
+    ua.send("k", x)
+    ua.send("v", x)
+    out = ua.attend()
+    ref = attention_per_head_ref(*(x.permute(0, 2, 1, 3),) * 3, sage.MODE_BF16,
+                                 torch.empty(1, 4, 8, 16, dtype=torch.bfloat16))
+    assert torch.equal(out.view(torch.int16), ref.permute(0, 2, 1, 3).contiguous().view(torch.int16))
+    assert sent == [(1, 1, 4, 8, 16)] * 4                                             # q, k, v, O chunks
