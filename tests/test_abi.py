@@ -144,3 +144,27 @@ def test_host_chunk_rule():
     assert sage.host_chunk_heads(1, 30, 17776, 64) == 9           # 70 CTAs per head
     assert sage.host_chunk_heads(1, 2, 1024, 128) == 2            # capped at B*H
     assert sage.host_chunk_heads(1, 2, 1024, 96) == 0             # bad shape
+
+
+def test_binding_checks_what_the_c_abi_cannot_see():
+    """dtype, contiguity and shape of tensor arguments are checked before any device call (CPU tensors)."""
+    import torch
+    xq = torch.zeros(256, 256, dtype=torch.int8)
+    s = torch.zeros(2, 2, dtype=torch.float32)
+    with pytest.raises(ValueError, match="int8"):
+        sage.linear_w8a8(xq.float(), s, xq, s)
+    with pytest.raises(ValueError, match="contiguous"):
+        sage.linear_w8a8(xq.t(), s, xq, s)
+    with pytest.raises(ValueError, match="shape"):
+        sage.linear_w8a8(xq, torch.zeros(3, 2), xq, s)
+    with pytest.raises(ValueError, match="bfloat16"):
+        sage.linear_bf16(torch.zeros(4, 128), torch.zeros(128, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="shape"):
+        sage.linear_w8a16(torch.zeros(4, 256, dtype=torch.bfloat16), xq, s, bias=torch.zeros(3, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="shape"):
+        sage.dequant_blocks_2d(xq, torch.zeros(1, 2))
+    a = torch.zeros(1, 8, 4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="multiple"):
+        sage.ulysses_permute(a, torch.zeros_like(a), 1, 8, 4, 16, 3, 0)
+    with pytest.raises(ValueError, match=r"\[P\] side"):
+        sage.ulysses_permute(a, torch.zeros(10, dtype=torch.bfloat16), 1, 8, 4, 16, 2, 0)

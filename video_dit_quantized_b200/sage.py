@@ -107,6 +107,20 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _need(t, name, dtype, shape=None, optional=False):
+    """Checks a tensor argument the C ABI cannot see: dtype, contiguity, shape."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def _bhnd(t, name):
     if t.dim() != 4:
         raise ValueError(f"{name} must be [B, H, N, d]")
@@ -313,6 +327,11 @@ def linear_w8a8(xq, sx, wq, sw, bias=None, y=None, out_dtype=None, status=None, 
     import torch
     M, K = xq.shape
     N = wq.shape[0]
+    _need(xq, "xq", torch.int8, (M, K))
+    _need(wq, "wq", torch.int8, (N, K))
+    _need(sx, "sx", torch.float32, ((M + BLK - 1) // BLK, K // BLK))
+    _need(sw, "sw", torch.float32, ((N + BLK - 1) // BLK, K // BLK))
+    _need(bias, "bias", torch.bfloat16, (N,), optional=True)
     if out_dtype is None:
         out_dtype = torch.bfloat16 if y is None else y.dtype
     if y is None:
@@ -329,6 +348,9 @@ def dequant_blocks_2d(codes, scales, out=None, stream=None):
     """int8 codes [R, K] + block scales -> bf16 [R, K] = bf16(scale * code)."""
     import torch
     R, K = codes.shape
+    _need(codes, "codes", torch.int8, (R, K))
+    _need(scales, "scales", torch.float32, ((R + BLK - 1) // BLK, K // BLK))
+    _need(out, "out", torch.bfloat16, (R, K), optional=True)
     if out is None:
         out = torch.empty((R, K), dtype=torch.bfloat16, device=codes.device)
     _check(LIB.sage_dequant_blocks_2d(_ptr(codes), _ptr(scales), R, K, _ptr(out), _stream(stream)),
@@ -341,6 +363,9 @@ def linear_bf16(x, w, bias=None, y=None, out_dtype=None, status=None, stream=Non
     import torch
     M, K = x.shape
     N = w.shape[0]
+    _need(x, "x", torch.bfloat16, (M, K))
+    _need(w, "w", torch.bfloat16, (N, K))
+    _need(bias, "bias", torch.bfloat16, (N,), optional=True)
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
     if status is None:
@@ -356,6 +381,10 @@ def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, s
     import torch
     M, K = x.shape
     N = wq.shape[0]
+    _need(x, "x", torch.bfloat16, (M, K))
+    _need(wq, "wq", torch.int8, (N, K))
+    _need(sw, "sw", torch.float32, ((N + BLK - 1) // BLK, K // BLK))
+    _need(bias, "bias", torch.bfloat16, (N,), optional=True)
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
     if status is None:
@@ -381,6 +410,18 @@ def host_chunk_heads(B: int, H: int, N: int, d: int) -> int:
 def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, chunk_rows: int = 0,
                     base_rows: int = 0, stream=None):
     """Row permutation between the Ulysses layouts (see include/sage.h); dst is filled and returned."""
+    import torch
+    _need(src, "src", torch.bfloat16)
+    _need(dst, "dst", torch.bfloat16)
+    if P < 1 or H % P:
+        raise ValueError(f"H={H} must be a multiple of P={P}")
+    dense = B * (H // P) * Nl                     # rows of one [P] chunk
+    p_side_rows = base_rows + (P - 1) * (chunk_rows or dense) + dense
+    chunked, flat = (dst, src) if op in (ULYSSES_SEND_QKV, ULYSSES_SEND_O) else (src, dst)
+    if flat.numel() < B * Nl * H * d:
+        raise ValueError("the [B, ...] side holds fewer than B * Nl * H rows of d values")
+    if chunked.numel() < p_side_rows * d:
+        raise ValueError("the [P] side is smaller than base_rows + (P - 1) * chunk_rows + one chunk")
     _check(LIB.sage_ulysses_permute(_ptr(src), _ptr(dst), B, Nl, H, d, P, op, int(chunk_rows), int(base_rows),
                                     _stream(stream)), "sage_ulysses_permute")
     return dst
