@@ -168,3 +168,12 @@ def test_binding_checks_what_the_c_abi_cannot_see():
         sage.ulysses_permute(a, torch.zeros_like(a), 1, 8, 4, 16, 3, 0)
     with pytest.raises(ValueError, match=r"\[P\] side"):
         sage.ulysses_permute(a, torch.zeros(10, dtype=torch.bfloat16), 1, 8, 4, 16, 2, 0)
+
+
+def test_attn_fwd_binding_checks():
+    import torch
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="bfloat16"):
+        sage.attn_fwd(q, q.float(), q, sage.MODE_BF16)
+    with pytest.raises(ValueError, match="shape"):
+        sage.attn_fwd(q, q, torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16), sage.MODE_BF16)

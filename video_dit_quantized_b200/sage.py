@@ -209,6 +209,8 @@ def attn_fwd(q, k, v, mode: int, o=None, workspace=None, stream=None):
     """Full-sequence self-attention through sage_attn_fwd; returns bf16 O [B,H,N,d]."""
     import torch
     B, H, N, d = _bhnd(q, "q")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(t, name, torch.bfloat16, (B, H, N, d), optional=name == "o")
     if o is None:
         o = torch.empty_like(q)
     if workspace is None:
