@@ -634,19 +634,16 @@ cudaError_t launch_linear_w8a8(const int8_t* xq, const float* sx, const int8_t* 
       !encode_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static int configured_dev = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes fa;
   if ((e = cudaFuncGetAttributes(&fa, linear_w8a8_kernel)) != cudaSuccess) return e;
   if (fa.numRegs * kThreads < 128 * REGS_LOW + 256 * REGS_HIGH) return cudaErrorInvalidConfiguration;
-  if (configured_dev != dev) {
-    if ((e = cudaFuncSetAttribute(linear_w8a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
-        cudaSuccess)
-      return e;
-    configured_dev = dev;
-  }
+  // set on every launch (per device, thread-safe; allowed during stream capture)
+  if ((e = cudaFuncSetAttribute(linear_w8a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+      cudaSuccess)
+    return e;
   int sms = 0;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   LinParams prm;
@@ -689,16 +686,12 @@ cudaError_t launch_linear_bf16(const void* x, const void* w, const void* bias, v
       !encode_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, bf16g::BK, bf16g::BN,
                       CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static int configured_dev = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_dev != dev) {
-    if ((e = cudaFuncSetAttribute(linear_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bf16g::SMEM_BYTES)) !=
-        cudaSuccess)
-      return e;
-    configured_dev = dev;
-  }
+  if ((e = cudaFuncSetAttribute(linear_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bf16g::SMEM_BYTES)) !=
+      cudaSuccess)
+    return e;
   int sms = 0;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   Bf16Params prm;
