@@ -114,6 +114,25 @@ def rank_workload(w, rank: int):
     return w.with_seed(w.seed + rank)
 
 
+# Exponentials per clock per SM: the SFU's ex2 rate (16 results/clk/SM; a microbenchmark with two issuing
+# warps per sub-partition measured 3.9 per clock per sub-partition).
+SFU_EX2_PER_CLK_PER_SM = 16.0
+
+
+def sfu_cap_tflops(d: int, sms: int, sm_mhz):
+    """The attention FLOP rate one ex2 per score allows: a call does 4*N^2*d FLOPs over N^2 exponentials,
+    so 4*d FLOPs per SFU result.  None without a clock reading."""
+    if not sm_mhz:
+        return None
+    return 4.0 * d * SFU_EX2_PER_CLK_PER_SM * sms * float(sm_mhz) * 1e6 / 1e12
+
+
+def sfu_cap(d: int, sms: int, sm_mhz, achieved: float):
+    cap = sfu_cap_tflops(d, sms, sm_mhz)
+    return {"tflops": cap, "frac": (achieved / cap) if cap else None,
+            "basis": "one ex2 per score at 16 results/clk/SM and the median SM clock"}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -408,7 +427,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_basis": f"{'2x ' if ratio == 2 else ''}bf16_tflops_sustained ({src})",
-                     "frac_of_datasheet_4500": achieved / (4500.0 if ratio == 2 else 2250.0)},
+                     "frac_of_datasheet_4500": achieved / (4500.0 if ratio == 2 else 2250.0),
+                     "sfu_cap": sfu_cap(w.d, probe["sms"], clocks["sm_mhz"], achieved)},
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

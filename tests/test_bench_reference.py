@@ -33,3 +33,16 @@ def test_linear_reference_line():
     assert KEYS <= set(d), KEYS - set(d)
     assert d["impl"] == "reference" and d["unit"] == "TOPS" and d["value"] > 0
     assert d["config"]["M"] == 333 and d["config"]["K"] == 512
+
+
+def test_sfu_cap_arithmetic():
+    """4*d FLOPs per exponential at 16 results/clk/SM: 2.38 PFLOP/s at d = 128, 148 SMs, 1965 MHz."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert abs(bench.sfu_cap_tflops(128, 148, 1965.0) - 4 * 128 * 16 * 148 * 1965e6 / 1e12) < 1e-9
+    assert 2380 < bench.sfu_cap_tflops(128, 148, 1965.0) < 2385
+    assert bench.sfu_cap_tflops(64, 148, 1965.0) * 2 == bench.sfu_cap_tflops(128, 148, 1965.0)
+    assert bench.sfu_cap_tflops(128, 148, None) is None
+    c = bench.sfu_cap(128, 148, 1965.0, 1416.2)
+    assert abs(c["frac"] - 1416.2 / c["tflops"]) < 1e-12
+    assert bench.sfu_cap(128, 148, None, 1416.2)["frac"] is None
