@@ -251,10 +251,17 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
     return SAGE_ELAUNCH;
   }
   // inputs of chunk i land (s_in) -> its attention runs (stream) -> its output leaves (s_out)
-  cudaEvent_t ev_start, ev_in, ev_done;
-  cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
-  cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
-  cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+  cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_done = nullptr;
+  if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) != cudaSuccess) {
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (ev_in) cudaEventDestroy(ev_in);
+    if (ev_done) cudaEventDestroy(ev_done);
+    cudaStreamDestroy(s_in);
+    cudaStreamDestroy(s_out);
+    return SAGE_ELAUNCH;
+  }
   // copies may not start before earlier work on the caller's stream
   cudaEventRecord(ev_start, st);
   cudaStreamWaitEvent(s_in, ev_start, 0);
