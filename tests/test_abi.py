@@ -177,3 +177,17 @@ def test_attn_fwd_binding_checks():
         sage.attn_fwd(q, q.float(), q, sage.MODE_BF16)
     with pytest.raises(ValueError, match="shape"):
         sage.attn_fwd(q, q, torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16), sage.MODE_BF16)
+
+
+def test_host_tensors_are_refused_for_device_arguments():
+    """The C ABI cannot tell a host address from a device one; the binding refuses CPU tensors (CPU test)."""
+    import torch
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="not a CUDA tensor"):
+        sage.attn_fwd(q, q, q, sage.MODE_BF16, workspace=torch.zeros(256, dtype=torch.uint8))
+    x = torch.zeros(256, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="not a CUDA tensor"):
+        sage.quantize_blocks_2d(x, torch.zeros(256, 256, dtype=torch.int8), torch.zeros(2, 2))
+    a = torch.zeros(1, 8, 4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="not a CUDA tensor"):
+        sage.ulysses_permute(a, torch.zeros_like(a), 1, 8, 4, 16, 2, 0)

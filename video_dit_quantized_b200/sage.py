@@ -101,6 +101,16 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _dptr(t):
+    """Device pointer of a CUDA tensor (None stays None).  The C ABI takes device pointers and cannot tell a
+    host address from a device one, so a host tensor is refused here instead of being read by a kernel."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("a tensor passed for device memory is not a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def _stream(stream=None):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -166,9 +176,9 @@ def quantize_qk(q, k, v, stream=None, q_per_token: bool = False):
     )
     nscr = prepass_scratch_bytes(B, H, N, d)
     scratch = torch.empty(max(nscr, 256), dtype=torch.uint8, device=dev)
-    _check(LIB.sage_quantize_qk_ex(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, 1 if q_per_token else BLK,
-                                   _ptr(out["q_i8"]), _ptr(out["q_scale"]), _ptr(out["k_i8"]), _ptr(out["k_scale"]),
-                                   _ptr(out["k_mean"]), _ptr(out["v_f8t"]), _ptr(out["v_scale"]), _ptr(scratch),
+    _check(LIB.sage_quantize_qk_ex(_dptr(q), _dptr(k), _dptr(v), B, H, N, d, 1 if q_per_token else BLK,
+                                   _dptr(out["q_i8"]), _dptr(out["q_scale"]), _dptr(out["k_i8"]), _dptr(out["k_scale"]),
+                                   _dptr(out["k_mean"]), _dptr(out["v_f8t"]), _dptr(out["v_scale"]), _dptr(scratch),
                                    scratch.numel(), _stream(stream)), "sage_quantize_qk_ex")
     out["_scratch"] = scratch
     out["_q_per_token"] = bool(q_per_token)
@@ -184,9 +194,9 @@ def quantize_qk_noalloc(q, k, v, out: dict, stream=None) -> int:
     caller-allocated outputs with the keys and shapes quantize_qk returns.
     Returns the status code (SAGE_EWORKSPACE if the problem exceeds the array)."""
     B, H, N, d = _bhnd(q, "q")
-    return int(LIB.sage_quantize_qk_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(out["q_i8"]),
-                                            _ptr(out["q_scale"]), _ptr(out["k_i8"]), _ptr(out["k_scale"]),
-                                            _ptr(out["k_mean"]), _ptr(out["v_f8t"]), _ptr(out["v_scale"]),
+    return int(LIB.sage_quantize_qk_noalloc(_dptr(q), _dptr(k), _dptr(v), B, H, N, d, _dptr(out["q_i8"]),
+                                            _dptr(out["q_scale"]), _dptr(out["k_i8"]), _dptr(out["k_scale"]),
+                                            _dptr(out["k_mean"]), _dptr(out["v_f8t"]), _dptr(out["v_scale"]),
                                             _stream(stream)))
 
 
@@ -199,9 +209,9 @@ def attn_quantized(pre: dict, N: int, o=None, status=None, stream=None):
     if status is None:
         status = torch.zeros(64, dtype=torch.int32, device=o.device)
     gran = 1 if pre.get("_q_per_token", False) else BLK
-    _check(LIB.sage_attn_quantized_ex(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]),
-                                      _ptr(pre["k_scale"]), _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o), B, H, N,
-                                      d, gran, _ptr(status), _stream(stream)), "sage_attn_quantized_ex")
+    _check(LIB.sage_attn_quantized_ex(_dptr(pre["q_i8"]), _dptr(pre["q_scale"]), _dptr(pre["k_i8"]),
+                                      _dptr(pre["k_scale"]), _dptr(pre["v_f8t"]), _dptr(pre["v_scale"]), _dptr(o), B, H, N,
+                                      d, gran, _dptr(status), _stream(stream)), "sage_attn_quantized_ex")
     return o
 
 
@@ -215,7 +225,7 @@ def attn_fwd(q, k, v, mode: int, o=None, workspace=None, stream=None):
         o = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(B, H, N, d, mode, q.device)
-    _check(LIB.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(mode), _ptr(workspace),
+    _check(LIB.sage_attn_fwd(_dptr(q), _dptr(k), _dptr(v), _dptr(o), B, H, N, d, int(mode), _dptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)), "sage_attn_fwd")
     return o
 
@@ -236,8 +246,8 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, c
     if workspace is None:
         workspace = alloc_workspace(1, chunk, N, d, mode)
     qd, kd, vd, od = staging
-    _check(LIB.sage_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), B, H, N, d, int(mode), _ptr(qd),
-                                  _ptr(kd), _ptr(vd), _ptr(od), _ptr(workspace),
+    _check(LIB.sage_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), B, H, N, d, int(mode), _dptr(qd),
+                                  _dptr(kd), _dptr(vd), _dptr(od), _dptr(workspace),
                                   workspace.numel() * workspace.element_size(), int(chunk), _stream(stream)),
            "sage_attn_fwd_host")
     return o_h
@@ -249,7 +259,7 @@ def error_stats(a, b, stream=None):
     B, H, N, d = _bhnd(a, "a")
     stats = torch.empty((B * H, 4), dtype=torch.float64, device=a.device)
     scratch = torch.empty(max(int(LIB.sage_error_scratch_bytes(B, H)), 16), dtype=torch.uint8, device=a.device)
-    _check(LIB.sage_attn_error_stats(_ptr(a), _ptr(b), B, H, N, d, _ptr(stats), _ptr(scratch), scratch.numel(),
+    _check(LIB.sage_attn_error_stats(_dptr(a), _dptr(b), B, H, N, d, _dptr(stats), _dptr(scratch), scratch.numel(),
                                      _stream(stream)), "sage_attn_error_stats")
     return stats
 
@@ -319,7 +329,7 @@ def quantize_blocks_2d(x, codes=None, scales=None, stream=None):
         codes = torch.empty((R, K), dtype=torch.int8, device=x.device)
     if scales is None:
         scales = torch.empty(((R + BLK - 1) // BLK, K // BLK), dtype=torch.float32, device=x.device)
-    _check(LIB.sage_quantize_blocks_2d(_ptr(x), R, K, _ptr(codes), _ptr(scales), _stream(stream)),
+    _check(LIB.sage_quantize_blocks_2d(_dptr(x), R, K, _dptr(codes), _dptr(scales), _stream(stream)),
            "sage_quantize_blocks_2d")
     return codes, scales
 
@@ -341,8 +351,8 @@ def linear_w8a8(xq, sx, wq, sw, bias=None, y=None, out_dtype=None, status=None, 
     if status is None:
         status = torch.zeros(64, dtype=torch.int32, device=xq.device)
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
-    _check(LIB.sage_linear_w8a8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M, N, K,
-                                _ptr(status), _stream(stream)), "sage_linear_w8a8")
+    _check(LIB.sage_linear_w8a8(_dptr(xq), _dptr(sx), _dptr(wq), _dptr(sw), _dptr(bias), _dptr(y), code, M, N, K,
+                                _dptr(status), _stream(stream)), "sage_linear_w8a8")
     return y
 
 
@@ -355,7 +365,7 @@ def dequant_blocks_2d(codes, scales, out=None, stream=None):
     _need(out, "out", torch.bfloat16, (R, K), optional=True)
     if out is None:
         out = torch.empty((R, K), dtype=torch.bfloat16, device=codes.device)
-    _check(LIB.sage_dequant_blocks_2d(_ptr(codes), _ptr(scales), R, K, _ptr(out), _stream(stream)),
+    _check(LIB.sage_dequant_blocks_2d(_dptr(codes), _dptr(scales), R, K, _dptr(out), _stream(stream)),
            "sage_dequant_blocks_2d")
     return out
 
@@ -373,7 +383,7 @@ def linear_bf16(x, w, bias=None, y=None, out_dtype=None, status=None, stream=Non
     if status is None:
         status = torch.zeros(64, dtype=torch.int32, device=x.device)
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
-    _check(LIB.sage_linear_bf16(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), code, M, N, K, _ptr(status),
+    _check(LIB.sage_linear_bf16(_dptr(x), _dptr(w), _dptr(bias), _dptr(y), code, M, N, K, _dptr(status),
                                 _stream(stream)), "sage_linear_bf16")
     return y
 
@@ -395,8 +405,8 @@ def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, s
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
-    _check(LIB.sage_linear_w8a16(_ptr(x), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M, N, K, _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)),
+    _check(LIB.sage_linear_w8a16(_dptr(x), _dptr(wq), _dptr(sw), _dptr(bias), _dptr(y), code, M, N, K, _dptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _dptr(status), _stream(stream)),
            "sage_linear_w8a16")
     return y
 
@@ -424,14 +434,14 @@ def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, 
         raise ValueError("the [B, ...] side holds fewer than B * Nl * H rows of d values")
     if chunked.numel() < p_side_rows * d:
         raise ValueError("the [P] side is smaller than base_rows + (P - 1) * chunk_rows + one chunk")
-    _check(LIB.sage_ulysses_permute(_ptr(src), _ptr(dst), B, Nl, H, d, P, op, int(chunk_rows), int(base_rows),
+    _check(LIB.sage_ulysses_permute(_dptr(src), _dptr(dst), B, Nl, H, d, P, op, int(chunk_rows), int(base_rows),
                                     _stream(stream)), "sage_ulysses_permute")
     return dst
 
 
 def status(workspace, stream=None) -> int:
     """Reads and clears the device status word (synchronises the stream); returns a status code."""
-    return int(LIB.sage_status(_ptr(workspace), _stream(stream)))
+    return int(LIB.sage_status(_dptr(workspace), _stream(stream)))
 
 
 def layer_schedule(num_layers: int, full_precision_layers) -> list[int]:
@@ -456,7 +466,7 @@ def dbg_qk_tiles(q_i8, k_i8, N: int, tiles, stream=None):
     B, H, _, d = q_i8.shape
     tl = torch.tensor(tiles, dtype=torch.int32, device=q_i8.device).reshape(-1, 4).contiguous()
     out = torch.empty((tl.shape[0], BLK, BLK), dtype=torch.int32, device=q_i8.device)
-    _check(LIB.sage_dbg_qk_tiles(_ptr(q_i8), _ptr(k_i8), B, H, N, d, _ptr(tl), tl.shape[0], _ptr(out),
+    _check(LIB.sage_dbg_qk_tiles(_dptr(q_i8), _dptr(k_i8), B, H, N, d, _dptr(tl), tl.shape[0], _dptr(out),
                                  _stream(stream)), "sage_dbg_qk_tiles")
     return out
 
@@ -465,7 +475,7 @@ def dbg_pv_tile(p, vt, mode: int, stream=None):
     import torch
     d = vt.shape[0] if mode == MODE_INT8_FP8 else vt.shape[1]
     out = torch.empty((BLK, d), dtype=torch.float32, device=p.device)
-    _check(LIB.sage_dbg_pv_tile(_ptr(p), _ptr(vt), d, int(mode), _ptr(out), _stream(stream)), "sage_dbg_pv_tile")
+    _check(LIB.sage_dbg_pv_tile(_dptr(p), _dptr(vt), d, int(mode), _dptr(out), _stream(stream)), "sage_dbg_pv_tile")
     return out
 
 
@@ -473,7 +483,7 @@ def dbg_qk_bf16_tile(q, k, stream=None):
     import torch
     d = q.shape[1]
     out = torch.empty((BLK, BLK), dtype=torch.float32, device=q.device)
-    _check(LIB.sage_dbg_qk_bf16_tile(_ptr(q), _ptr(k), d, _ptr(out), _stream(stream)), "sage_dbg_qk_bf16_tile")
+    _check(LIB.sage_dbg_qk_bf16_tile(_dptr(q), _dptr(k), d, _dptr(out), _stream(stream)), "sage_dbg_qk_bf16_tile")
     return out
 
 
@@ -484,8 +494,8 @@ def dbg_linear_forced_timeout(xq, sx, wq, sw, status, timeout_cycles: int, bias=
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
-    _check(LIB.sage_dbg_linear_forced_timeout(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), code, M,
-                                              N, K, _ptr(status), int(timeout_cycles), _stream(stream)),
+    _check(LIB.sage_dbg_linear_forced_timeout(_dptr(xq), _dptr(sx), _dptr(wq), _dptr(sw), _dptr(bias), _dptr(y), code, M,
+                                              N, K, _dptr(status), int(timeout_cycles), _stream(stream)),
            "sage_dbg_linear_forced_timeout")
     return y
 
@@ -497,7 +507,7 @@ def dbg_linear_bf16_forced_timeout(x, w, status, timeout_cycles: int, bias=None,
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     code = DTYPE_F32 if y.dtype == torch.float32 else DTYPE_BF16
-    _check(LIB.sage_dbg_linear_bf16_forced_timeout(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), code, M, N, K, _ptr(status),
+    _check(LIB.sage_dbg_linear_bf16_forced_timeout(_dptr(x), _dptr(w), _dptr(bias), _dptr(y), code, M, N, K, _dptr(status),
                                                    int(timeout_cycles), _stream(stream)),
            "sage_dbg_linear_bf16_forced_timeout")
     return y
@@ -512,7 +522,7 @@ def dbg_mma_peak(kind: int, n: int = 256, iters: int = 4000, stream=None) -> dic
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     cycles = torch.zeros(sms, dtype=torch.int64, device="cuda")
     status = torch.zeros(64, dtype=torch.int32, device="cuda")
-    _check(LIB.sage_dbg_mma_peak(int(kind), int(n), int(iters), _ptr(cycles), sms, _ptr(status), _stream(stream)),
+    _check(LIB.sage_dbg_mma_peak(int(kind), int(n), int(iters), _dptr(cycles), sms, _dptr(status), _stream(stream)),
            "sage_dbg_mma_peak")
     torch.cuda.synchronize()
     if int(status[0].item()) != 0:
@@ -527,8 +537,8 @@ def dbg_attn_forced_timeout(pre: dict, N: int, status, timeout_cycles: int, o=No
     B, H, _, d = pre["q_i8"].shape
     if o is None:
         o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=pre["q_i8"].device)
-    _check(LIB.sage_dbg_attn_forced_timeout(_ptr(pre["q_i8"]), _ptr(pre["q_scale"]), _ptr(pre["k_i8"]),
-                                            _ptr(pre["k_scale"]), _ptr(pre["v_f8t"]), _ptr(pre["v_scale"]), _ptr(o),
-                                            B, H, N, d, _ptr(status), int(timeout_cycles), _stream(stream)),
+    _check(LIB.sage_dbg_attn_forced_timeout(_dptr(pre["q_i8"]), _dptr(pre["q_scale"]), _dptr(pre["k_i8"]),
+                                            _dptr(pre["k_scale"]), _dptr(pre["v_f8t"]), _dptr(pre["v_scale"]), _dptr(o),
+                                            B, H, N, d, _dptr(status), int(timeout_cycles), _stream(stream)),
            "sage_dbg_attn_forced_timeout")
     return o
