@@ -191,3 +191,38 @@ def test_host_tensors_are_refused_for_device_arguments():
     a = torch.zeros(1, 8, 4, 16, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="not a CUDA tensor"):
         sage.ulysses_permute(a, torch.zeros_like(a), 1, 8, 4, 16, 2, 0)
+
+
+def _header_decls():
+    """(name, return type, [parameter types]) of every function in include/sage.h."""
+    import re
+    txt = re.sub(r"/\*.*?\*/", "", open(sage.HEADER).read(), flags=re.S)
+    txt = re.sub(r"//[^\n]*", "", txt)
+    out = []
+    for m in re.finditer(r"^\s*((?:const\s+)?[A-Za-z_][\w\s\*]*?)\b([a-z_][a-z0-9_]*)\s*\(([^)]*)\)\s*;", txt, flags=re.M):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        types = [] if params in ("", "void") else [re.sub(r"\s*\b\w+$", "", p.strip()) for p in params.split(",")]
+        out.append((name, ret, types))
+    return out
+
+
+def _ctype(c: str):
+    c = " ".join(c.replace("*", " * ").split())
+    if c == "const char *":
+        return ctypes.c_char_p
+    if "*" in c:
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "long long": ctypes.c_longlong,
+            "double": ctypes.c_double}[c.replace("const ", "")]
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes prototype has the header's argument count and kinds (a mismatch would pass garbage
+    pointers to the device) and its return type."""
+    decls = _header_decls()
+    assert {n for n, _, _ in decls} == EXPECTED
+    for name, ret, params in decls:
+        f = getattr(sage.LIB, name)
+        assert f.argtypes is not None, name
+        assert [a for a in f.argtypes] == [_ctype(p) for p in params], name
+        assert f.restype == _ctype(ret), name
