@@ -90,3 +90,18 @@ def test_zero_k_channel_bf16_rounding_and_determinism():
     assert all(np.array_equal(a, b) for a, b in zip((q, k, v), again))
     other = synth.qkv_numpy(w.with_seed(6))
     assert not np.array_equal(q, other[0])
+
+
+def test_linear_operands_recipe():
+    """X ~ N(0,1) with round(0.01 K) outlier channels x20, W ~ N(0, 1/K), bias ~ 0.02 N(0,1)."""
+    lw = synth.LinearWorkload("recipe_lin", 4096, 384, 1024, seed=9)
+    assert lw.n_outlier == 10
+    x, wt, b = (synth.bf16_bits_to_f32(a).astype(np.float64) for a in synth.linear_numpy(lw))
+    col_std = x.std(axis=0)
+    out = col_std > 5.0
+    assert out.sum() == 10
+    assert np.all(np.abs(col_std[out] - 20.0) < 1.5) and np.all(np.abs(col_std[~out] - 1.0) < 0.1)
+    assert abs(x[:, ~out].mean()) < 5 / math.sqrt(x[:, ~out].size)
+    assert abs(wt.std() * math.sqrt(lw.K) - 1.0) < 0.01
+    assert abs(b.std() / 0.02 - 1.0) < 0.15          # 384 draws
+    assert np.array_equal(synth.linear_numpy(lw)[0], synth.linear_numpy(lw)[0])
