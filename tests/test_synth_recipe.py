@@ -105,3 +105,13 @@ def test_linear_operands_recipe():
     assert abs(wt.std() * math.sqrt(lw.K) - 1.0) < 0.01
     assert abs(b.std() / 0.02 - 1.0) < 0.15          # 384 draws
     assert np.array_equal(synth.linear_numpy(lw)[0], synth.linear_numpy(lw)[0])
+
+
+def test_sampled_rows_cover_the_edges():
+    """Parity samples always hold row 0, row N-1 and the first row of the tail tile; sorted, distinct."""
+    for seed, N, n in [(0, 75600, 48), (3, 17776, 16), (5, 129, 8), (1, 100, 500), (2, 1, 4)]:
+        rows = synth.sample_rows(seed, N, n)
+        assert len(rows) == min(n, N)
+        assert np.all(np.diff(rows) > 0) and rows[0] >= 0 and rows[-1] < N
+        assert {0, N - 1, (N - 1) // 128 * 128} <= set(rows.tolist())
+    assert np.array_equal(synth.sample_rows(7, 5000, 20), synth.sample_rows(7, 5000, 20))
