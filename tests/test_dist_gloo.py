@@ -105,9 +105,10 @@ def _ulysses_rank(rank, world, port, result_q):
         dist.destroy_process_group()
 
 
-def test_ulysses_exchange_two_gloo_ranks():
-    """Two CPU ranks run the Ulysses exchange around a per-head reference attention; each rank's
-    output slice equals single-process attention on the whole sequence, bit for bit."""
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_exchange_gloo_ranks(world):
+    """Two or four CPU ranks run the Ulysses exchange around a per-head reference attention; each
+    rank's output slice equals single-process attention on the whole sequence, bit for bit."""
     import multiprocessing as mp
     import socket
 
@@ -116,14 +117,14 @@ def test_ulysses_exchange_two_gloo_ranks():
         port = s.getsockname()[1]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_ulysses_rank, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_ulysses_rank, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
-    results = dict(q.get(timeout=5) for _ in range(2))
-    assert results == {0: True, 1: True}
+    results = dict(q.get(timeout=5) for _ in range(world))
+    assert results == {r: True for r in range(world)}
 
 
 def test_ulysses_host_checks():
