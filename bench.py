@@ -18,6 +18,12 @@ runs on them, and O goes back.  The total problem is fixed (strong scaling);
 value = the full layer's attention FLOPs / max-over-ranks time.  On one GPU
 the exchange is a single-rank NCCL all-to-all (a local copy).
 
+`--op stack` times the layer-selective stack as one unit: 40 consecutive
+attention calls at B=1, H=40, N=32760, d=128 with seed = layer index, the
+modes from attn_layer_schedule (layers 0, 8, 16, 24, 32 in BF16, the rest
+INT8/FP8, prepass included); one step = the whole stack.  It also times the
+same 40 calls all in BF16 for comparison and splits the time by mode.
+
 `--op linear` times the W8A8 linear layer with 128 x 128 block scales
 instead (one step = block-quantize the activations X [M, K] + the block-scaled
 INT8 GEMM against pre-quantized weights W [N, K], plus bias), at the
@@ -84,7 +90,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3, help="end-to-end steps (at least 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4096)
-    ap.add_argument("--op", default="attention", choices=["attention", "linear", "ulysses"])
+    ap.add_argument("--op", default="attention", choices=["attention", "linear", "ulysses", "stack"])
     ap.add_argument("--linear-workload", default="wan14b_720p_proj", choices=sorted(synth.LINEAR_WORKLOADS))
     ap.add_argument("--linear-mode", default="w8a8", choices=["w8a8", "w8a16", "bf16"])
     return ap.parse_args()
@@ -241,7 +247,8 @@ def run_reference(args, rank, world):
     if args.op == "linear":
         run_reference_linear(args, rank, world)
         return
-    w = workload(args)
+    # the stack's calls all have the layer-stack shape; one sampled call per step stands for them
+    w = synth.WORKLOADS["layer_stack"] if args.op == "stack" else workload(args)
     if rank != 0:
         return
     rows = max(64, args.cpu_rows // 8)
@@ -669,11 +676,133 @@ def run_ulysses(args, rank, world, local_rank):
     }), flush=True)
 
 
+def run_stack(args, rank, world, local_rank):
+    """The 40-call layer-selective stack (one step = all 40 calls, each with its own seeded inputs)."""
+    import torch
+    import torch.distributed as dist
+    from video_dit_quantized_b200 import sage
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = synth.WORKLOADS["layer_stack"]
+    L = synth.LAYER_STACK_LAYERS
+    modes = sage.layer_schedule(L, synth.LAYER_STACK_FULL_PRECISION)
+    host, inputs = [], []
+    for layer in range(L):
+        # every rank runs its own independent stack: layer seeds offset by rank
+        h = synth.qkv_torch(base.with_seed(layer + rank * L), pin=True)
+        host.append(h)
+        inputs.append(tuple(t.to(dev, non_blocking=True) for t in h))
+    o = torch.empty_like(inputs[0][0])
+    ws = sage.alloc_workspace(base.B, base.H, base.N, base.d, sage.MODE_INT8_FP8, dev)
+    stream = torch.cuda.current_stream()
+    sp = sage._stream(stream)
+    P = sage._ptr
+    torch.cuda.synchronize()
+
+    def stack(layer_modes, evs=None):
+        for layer in range(L):
+            q, k, v = inputs[layer]
+            if evs:
+                evs[layer][0].record(stream)
+            rc = sage.LIB.sage_attn_fwd(P(q), P(k), P(v), P(o), base.B, base.H, base.N, base.d, layer_modes[layer],
+                                        P(ws), ws.numel(), sp)
+            if rc:
+                raise sage.SageError(rc, "sage_attn_fwd")
+            if evs:
+                evs[layer][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(layer_modes):
+        for _ in range(args.warmup):
+            stack(layer_modes)
+        torch.cuda.synchronize()
+        evs = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(2)) for _ in range(L)]
+               for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clk:
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for i in range(args.steps):
+                stack(layer_modes, evs[i])
+            t1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        st = sage.status(ws)
+        if st != sage.OK:
+            raise sage.SageError(st, "stack")
+        per_call = [[a.elapsed_time(b) for a, b in step] for step in evs]
+        return max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps, per_call, clk.summary()
+
+    ms, per_call, clocks = timed(modes)
+    ms_bf16, _, clocks_bf16 = timed([sage.MODE_BF16] * L)
+
+    # end to end: every layer's Q, K, V from pinned host memory through the public host-buffer call,
+    # its O back to pinned host memory
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    chunk = sage.host_chunk_heads(base.B, base.H, base.N, base.d)
+    ws_e2e = sage.alloc_workspace(1, chunk, base.N, base.d, sage.MODE_INT8_FP8, dev)
+    staging = tuple(torch.empty_like(o) for _ in range(4))
+
+    def e2e_stack():
+        for layer in range(L):
+            sage.attn_fwd_host(*host[layer], o_h, modes[layer], staging=staging, workspace=ws_e2e,
+                               chunk_heads=chunk, stream=stream)
+
+    e2e_stack()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_stack()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if rank != 0:
+        return
+    flops = L * base.flops
+    peaks, src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    by_mode = {}
+    for name, m, pk in (("int8_fp8", sage.MODE_INT8_FP8, 2.0 * sustained), ("bf16", sage.MODE_BF16, sustained)):
+        calls = [c for step in per_call for c, mm in zip(step, modes) if mm == m]
+        avg = statistics.mean(calls)
+        ach = base.flops / (avg * 1e-3) / 1e12
+        by_mode[name] = {"calls_per_stack": sum(1 for mm in modes if mm == m), "ms_per_call_mean": avg,
+                         "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                         "peak_basis": f"{'2x ' if m != sage.MODE_BF16 else ''}bf16_tflops_sustained ({src})"}
+    h2d = L * 3 * o.numel() * o.element_size()
+    d2h = L * o.numel() * o.element_size()
+    print(json.dumps({
+        "op": "layer_stack",
+        "metric": "attention TFLOPS per call (4*B*H*N^2*d), 40-layer selective stack",
+        "value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8/fp8e4m3 + bf16 layers (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": "layer_stack", "layers": L, "B": base.B, "H": base.H, "N": base.N, "d": base.d,
+                   "full_precision_layers": list(synth.LAYER_STACK_FULL_PRECISION), "seeds": "layer index",
+                   "parallelism": f"independent stacks x{world}",
+                   "l2": "every layer's inputs (1.0 GB) larger than L2; no flush"},
+        "by_mode": by_mode,
+        "all_bf16_stack": {"ms_per_step": ms_bf16, "tflops": flops / (ms_bf16 * 1e-3) / 1e12,
+                           "speedup_of_selective": ms_bf16 / ms, "clocks": clocks_bf16},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * sum(4 if m != sage.MODE_BF16 else 1 for m in modes),
+        "clocks": clocks,
+    }), flush=True)
+
+
 def main():
     args = parse()
     if args.steps is None:
         # a linear step is ~2.5 ms: 400 steps keep the timed region (and its clock samples) near a second
-        args.steps = 400 if args.op == "linear" else 20
+        args.steps = {"linear": 400, "stack": 3}.get(args.op, 20)
     args.e2e_steps = max(1, args.e2e_steps)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -697,6 +826,8 @@ def main():
     try:
         if args.op == "ulysses":
             run_ulysses(args, rank, world, local_rank)
+        elif args.op == "stack":
+            run_stack(args, rank, world, local_rank)
         elif args.op == "linear":
             run_linear(args, rank, world, local_rank)
         else:

@@ -125,8 +125,11 @@ int sage_quantize_qk(const void* q, const void* k, const void* v, int B, int H, 
  *    > SAGE_NOALLOC_SCRATCH_BYTES, e.g. B*H*ceil(N/128)*d above ~1.6M) are
  *    rejected with SAGE_EWORKSPACE before anything is launched.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, once per device, with that device current); make
- *    that first call before any stream capture.
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.  The address is cached with the id of the
+ *    CUDA context it belongs to; the first call in a new context (after
+ *    cudaDeviceReset, which also frees the array's old contents) looks it up
+ *    again, so that call too must come before any capture.
  *  - Every call shares the one array.  Calls whose kernels may overlap on the
  *    GPU (different streams, or several host threads) race on it and give
  *    wrong results: serialise them on one stream.  Each call overwrites every
@@ -142,8 +145,9 @@ int sage_quantize_qk_noalloc(const void* q, const void* k, const void* v, int B,
  * Attention over already-quantized operands (steps a5-a9): per 128x128 tile
  * S = Q_i8 K_i8^T in exact int32 (tcgen05 kind::i8), s = S * q_scale * k_scale
  * * log2(e)/sqrt(d), keys >= N masked, online softmax with p = 2^(s - m),
- * P8 = e4m3(p * 448) kept in tensor memory, O += P8 V8 (tcgen05 kind::f8f6f4,
- * fp32), O = O * v_scale / (448 * l) rounded to bf16.
+ * P8 = e4m3(p * 448) staged in shared memory (128-byte swizzled K-major tile),
+ * O += P8 V8 (tcgen05 kind::f8f6f4 from shared memory, fp32 in tensor
+ * memory), O = O * v_scale / (448 * l) rounded to bf16.
  * Operands as written by sage_quantize_qk; o is bf16 [B,H,N,d] (output).
  * status: a 256-byte device status region (e.g. the start of a workspace);
  * failures are OR-ed into its first word.
@@ -223,18 +227,32 @@ int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_
  * Deterministic (fixed summation order).  scratch: device buffer of
  * sage_error_scratch_bytes(B, H) bytes.  Asynchronous on `stream`.
  *
+ * sage_attn_rel_l2: the error of one layer at one iteration, the relative L2
+ * distance of a from b over every element of the layer (all B*H heads):
+ * out = sqrt(sum (a-b)^2 / sum b^2) as one fp64 value written to the device
+ * pointer `out` (0 when both sums are 0, +inf when only sum b^2 is).  The
+ * per-head sums are formed as in sage_attn_error_stats and added over the
+ * heads in ascending order on the device, so the result is deterministic.
+ * Same arguments, alignment, scratch and stream rules as
+ * sage_attn_error_stats; `out` must be 8-byte aligned.
+ *
  * sage_select_full_precision_layers: host layer_err [num_layers][num_iters]
- * (any per-layer, per-iteration error, e.g. the relative L2 error above);
- * writes, in ascending order, the layers whose mean error over the iterations
- * exceeds `threshold` to host layers_out[num_layers] and their count to
- * *n_out; the result feeds attn_layer_schedule.  SAGE_EINVAL on a non-finite
- * error or bad sizes.
+ * (any per-layer, per-iteration error, e.g. sage_attn_rel_l2's); writes, in
+ * ascending order, the layers kept at full precision to host
+ * layers_out[num_layers] and their count to *n_out; the result feeds
+ * attn_layer_schedule.  rule SAGE_SELECT_EVERY_ITERATION (the page's reading:
+ * the error is above `threshold` at every iteration) or SAGE_SELECT_MEAN (the
+ * mean error over the iterations is above it).  SAGE_EINVAL on a non-finite
+ * error, an unknown rule or bad sizes.
  */
+enum { SAGE_SELECT_EVERY_ITERATION = 0, SAGE_SELECT_MEAN = 1 };
 size_t sage_error_scratch_bytes(int B, int H);
 int sage_attn_error_stats(const void* a, const void* b, int B, int H, int N, int d, double* stats,
                           void* scratch, size_t scratch_bytes, void* stream);
+int sage_attn_rel_l2(const void* a, const void* b, int B, int H, int N, int d, double* out, void* scratch,
+                     size_t scratch_bytes, void* stream);
 int sage_select_full_precision_layers(const double* layer_err, int num_layers, int num_iters,
-                                      double threshold, int* layers_out, int* n_out);
+                                      double threshold, int rule, int* layers_out, int* n_out);
 
 /*
  * 8-bit linear layers with 128 x 128 block scales (TMAP write-up, "FFN
@@ -360,7 +378,9 @@ int sage_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int B, int H, int 
 
 /*
  * Diagnostic: one 128-row P.V product through the same operand path as the
- * attention kernels, with P written to tensor memory from registers.
+ * attention kernels: INT8_FP8 writes P from registers into the swizzled
+ * shared-memory tile and issues the shared-memory kind::f8f6f4 MMA; BF16
+ * writes P into tensor memory and issues the kind::f16 MMA with A there.
  * mode INT8_FP8: p (device, e4m3 [128,128]) times vt (device, e4m3 [d,128],
  *   key-contiguous) -> out fp32 [128,d] = sum_j p[i,j] * vt[c,j].
  * mode BF16: p (device, bf16 [128,128]) times vt (device, bf16 [128,d],

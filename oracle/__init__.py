@@ -78,6 +78,10 @@ def _load():
             lib.orc_dequant_blocks_2d.argtypes = [i8, f32, i32, i32, u16]
             lib.orc_layer_schedule.argtypes = [i32, P(i32), i32, i8]
             lib.orc_layer_schedule.restype = i32
+            lib.orc_rel_l2.argtypes = [u16, u16, i64]
+            lib.orc_rel_l2.restype = ctypes.c_double
+            lib.orc_select_layers.argtypes = [f64, i32, i32, ctypes.c_double, i32, P(i32)]
+            lib.orc_select_layers.restype = i32
             _lib = lib
     return _lib
 
@@ -270,3 +274,32 @@ def layer_schedule(num_layers: int, fp_layers) -> np.ndarray:
     if rc != 0:
         raise ValueError("layer index out of range")
     return modes
+
+
+# ---------------- f2: per-layer error and the full-precision layer set ----------------
+
+SELECT_EVERY_ITERATION = 0
+SELECT_MEAN = 1
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    """sqrt(sum (a-b)^2 / sum b^2) over every element of two bf16 arrays (uint16 bits), fp64 ascending sums."""
+    a = _c(a, np.uint16).ravel()
+    b = _c(b, np.uint16).ravel()
+    if a.size != b.size:
+        raise ValueError("a and b differ in size")
+    return float(_load().orc_rel_l2(_p(a, ctypes.c_uint16), _p(b, ctypes.c_uint16), a.size))
+
+
+def select_layers(err, threshold: float, rule: int = SELECT_EVERY_ITERATION) -> list[int]:
+    """Layers kept at full precision from err[layer][iteration] (rule 0: above the threshold at every
+    iteration; rule 1: mean above it)."""
+    e = np.ascontiguousarray(np.asarray(err, dtype=np.float64))
+    if e.ndim != 2:
+        raise ValueError("err must be [layers][iterations]")
+    out = np.zeros(max(e.shape[0], 1), dtype=np.int32)
+    n = _load().orc_select_layers(_p(e, ctypes.c_double), e.shape[0], e.shape[1], float(threshold), int(rule),
+                                  _p(out, ctypes.c_int))
+    if n < 0:
+        raise ValueError("bad error table or rule")
+    return out[:n].tolist()

@@ -508,3 +508,54 @@ int orc_layer_schedule(int num_layers, const int* fp_layers, int n_fp, int8_t* m
     for (int i = 0; i < n_fp; ++i) modes[fp_layers[i]] = 0;
     return 0;
 }
+
+/* ---------------- f2: per-layer error and the full-precision layer set ---------------- */
+
+/*
+ * Page 1, "Attention performance optimisation / Keeping video quality": the
+ * attention error of every layer was measured at every denoising iteration,
+ * and the layers whose error stayed large keep the original precision.
+ *
+ * The error of one layer at one iteration: the relative L2 distance of the
+ * quantized output a from the full-precision output b over every element of
+ * the layer's output (all heads), sqrt(sum (a - b)^2 / sum b^2), with both
+ * sums in fp64 in ascending element order.  b == 0 everywhere gives 0 when a
+ * is also 0 and +inf otherwise.
+ */
+double orc_rel_l2(const uint16_t* a, const uint16_t* b, long n) {
+    double num = 0.0, den = 0.0;
+    for (long i = 0; i < n; ++i) {
+        const double x = (double)bf16f(a[i]), y = (double)bf16f(b[i]);
+        const double diff = x - y;
+        num += diff * diff;
+        den += y * y;
+    }
+    if (den == 0.0) return num == 0.0 ? 0.0 : INFINITY;
+    return sqrt(num / den);
+}
+
+/*
+ * The full-precision set from the error table err[layer][iteration]:
+ *   rule 0: a layer whose error exceeds the threshold at EVERY iteration (the
+ *           page's "large at every iteration");
+ *   rule 1: a layer whose mean error over the iterations exceeds it.
+ * Writes the chosen layers in ascending order; returns how many, or -1 on a
+ * bad size, an unknown rule or a non-finite error.
+ */
+int orc_select_layers(const double* err, int num_layers, int num_iters, double threshold, int rule, int* out) {
+    if (num_layers < 0 || num_iters < 1 || (rule != 0 && rule != 1)) return -1;
+    int n = 0;
+    for (int l = 0; l < num_layers; ++l) {
+        int every = 1;
+        double sum = 0.0;
+        for (int i = 0; i < num_iters; ++i) {
+            const double e = err[(long)l * num_iters + i];
+            if (!isfinite(e)) return -1;
+            if (!(e > threshold)) every = 0;
+            sum += e;
+        }
+        const int pick = rule == 0 ? every : (sum / (double)num_iters > threshold);
+        if (pick) out[n++] = l;
+    }
+    return n;
+}

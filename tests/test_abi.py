@@ -15,6 +15,7 @@ EXPECTED = {
     "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
     "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
     "sage_ulysses_permute", "sage_host_chunk_heads", "sage_dbg_mma_peak", "sage_dbg_linear_bf16_forced_timeout",
+    "sage_attn_rel_l2",
 }
 
 
@@ -73,13 +74,33 @@ def test_strerror_covers_codes():
 
 
 def test_select_full_precision_layers_host():
+    import oracle
     err = [[0.01, 0.02], [0.30, 0.25], [0.05, 0.40], [0.2, 0.1]]
-    # means 0.015, 0.275, 0.225, 0.15
-    assert sage.select_full_precision_layers(err, 0.2) == [1, 2]
+    # above 0.2 at every iteration: layer 1 only; means 0.015, 0.275, 0.225, 0.15
+    assert sage.select_full_precision_layers(err, 0.2) == [1]
+    assert sage.select_full_precision_layers(err, 0.2, sage.SELECT_MEAN) == [1, 2]
     assert sage.select_full_precision_layers(err, 0.0) == [0, 1, 2, 3]
     assert sage.select_full_precision_layers(err, 1.0) == []
+    for rule in (sage.SELECT_EVERY_ITERATION, sage.SELECT_MEAN):
+        for thr in (0.0, 0.05, 0.1, 0.2, 0.25, 0.3, 1.0):
+            assert sage.select_full_precision_layers(err, thr, rule) == oracle.select_layers(err, thr, rule)
     with pytest.raises(sage.SageError):
         sage.select_full_precision_layers([[float("nan")]], 0.1)
+    with pytest.raises(sage.SageError):
+        sage.select_full_precision_layers(err, 0.1, 2)
+
+
+def test_rel_l2_argument_validation_runs_on_the_host():
+    lib = sage.LIB
+    fake = ctypes.c_void_p(1 << 20)
+    odd8 = ctypes.c_void_p((1 << 20) + 8)       # 8-byte aligned: allowed for out only
+    odd4 = ctypes.c_void_p((1 << 20) + 4)
+    nb = lib.sage_error_scratch_bytes(1, 2)
+    assert lib.sage_attn_rel_l2(fake, fake, 1, 2, 10, 128, odd4, fake, nb, None) == sage.EINVAL
+    assert lib.sage_attn_rel_l2(odd8, fake, 1, 2, 10, 128, fake, fake, nb, None) == sage.EINVAL
+    assert lib.sage_attn_rel_l2(fake, fake, 1, 2, 10, 12, fake, fake, nb, None) == sage.EINVAL
+    assert lib.sage_attn_rel_l2(fake, fake, 1, 2, 10, 128, fake, fake, nb - 8, None) == sage.EWORKSPACE
+    assert lib.sage_attn_rel_l2(None, fake, 1, 2, 10, 128, fake, fake, nb, None) == sage.EINVAL
 
 
 def test_linear_argument_validation_runs_on_the_host():

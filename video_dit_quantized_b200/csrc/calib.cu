@@ -10,7 +10,12 @@
 // Two kernels: per (head, slice) partial sums with a fixed per-thread order
 // and a fixed shared-memory tree, then per head the slices in ascending order,
 // so the result is deterministic.
-// sage_select_full_precision_layers: the selection rule, on the host.
+// sage_attn_rel_l2: the same partial sums, then one thread adds every head's
+// (a-b)^2 and b^2 slices in ascending order and writes sqrt(num / den).
+// sage_select_full_precision_layers: the selection rule, on the host: a layer
+// stays at full precision when its error is above the threshold at every
+// iteration (the page's "large in every iteration"), or, with the mean rule,
+// when its mean error over the iterations is.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -74,6 +79,29 @@ __global__ void err_final_kernel(const double* __restrict__ partial, int BH, dou
   stats[i] = sum;
 }
 
+// one thread: every head's slices in ascending order, then the relative L2 error
+__global__ void rel_l2_final_kernel(const double* __restrict__ partial, int BH, double* __restrict__ out) {
+  if (blockIdx.x != 0 || threadIdx.x != 0) return;
+  double num = 0.0, den = 0.0;
+  for (int bh = 0; bh < BH; ++bh)
+    for (int s = 0; s < kErrSlices; ++s) {
+      num += partial[((long long)bh * kErrSlices + s) * 4 + 0];
+      den += partial[((long long)bh * kErrSlices + s) * 4 + 1];
+    }
+  *out = den == 0.0 ? (num == 0.0 ? 0.0 : (double)INFINITY) : sqrt(num / den);
+}
+
+int check_err_args(const void* a, const void* b, int B, int H, int N, int d, const void* out, const void* scratch,
+                   size_t scratch_bytes) {
+  if (B < 1 || H < 1 || N < 1 || d < 8 || (d % 8) != 0) return SAGE_EINVAL;
+  if ((long long)B * H > 65535) return SAGE_EINVAL;
+  const void* ptrs[] = {a, b, out, scratch};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u) != 0) return SAGE_EINVAL;
+  if (scratch_bytes < (size_t)B * H * kErrSlices * 4 * sizeof(double)) return SAGE_EWORKSPACE;
+  return SAGE_OK;
+}
+
 }  // namespace
 }  // namespace sage
 
@@ -86,12 +114,8 @@ extern "C" size_t sage_error_scratch_bytes(int B, int H) {
 
 extern "C" int sage_attn_error_stats(const void* a, const void* b, int B, int H, int N, int d, double* stats,
                                      void* scratch, size_t scratch_bytes, void* stream) {
-  if (B < 1 || H < 1 || N < 1 || d < 8 || (d % 8) != 0) return SAGE_EINVAL;
-  if ((long long)B * H > 65535) return SAGE_EINVAL;
-  const void* ptrs[] = {a, b, stats, scratch};
-  for (const void* p : ptrs)
-    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u) != 0) return SAGE_EINVAL;
-  if (scratch_bytes < sage_error_scratch_bytes(B, H)) return SAGE_EWORKSPACE;
+  const int rc = check_err_args(a, b, B, H, N, d, stats, scratch, scratch_bytes);
+  if (rc != SAGE_OK) return rc;
   const int BH = B * H;
   const long long words = (long long)N * d / 8;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -102,19 +126,38 @@ extern "C" int sage_attn_error_stats(const void* a, const void* b, int B, int H,
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ELAUNCH;
 }
 
+extern "C" int sage_attn_rel_l2(const void* a, const void* b, int B, int H, int N, int d, double* out, void* scratch,
+                                size_t scratch_bytes, void* stream) {
+  if (out && (reinterpret_cast<uintptr_t>(out) & 7u) != 0) return SAGE_EINVAL;
+  // out needs only 8-byte alignment: check the others with a 16-byte aligned stand-in
+  const int rc = check_err_args(a, b, B, H, N, d, out ? scratch : nullptr, scratch, scratch_bytes);
+  if (rc != SAGE_OK) return rc;
+  const int BH = B * H;
+  const long long words = (long long)N * d / 8;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double* partial = static_cast<double*>(scratch);
+  err_partial_kernel<<<dim3(kErrSlices, BH), kErrThreads, 0, st>>>(static_cast<const uint4*>(a),
+                                                                   static_cast<const uint4*>(b), words, partial);
+  rel_l2_final_kernel<<<1, 32, 0, st>>>(partial, BH, out);
+  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ELAUNCH;
+}
+
 extern "C" int sage_select_full_precision_layers(const double* layer_err, int num_layers, int num_iters,
-                                                 double threshold, int* layers_out, int* n_out) {
+                                                 double threshold, int rule, int* layers_out, int* n_out) {
   if (num_layers < 0 || num_iters < 1 || !n_out || (num_layers > 0 && (!layer_err || !layers_out))) return SAGE_EINVAL;
+  if (rule != SAGE_SELECT_EVERY_ITERATION && rule != SAGE_SELECT_MEAN) return SAGE_EINVAL;
   int n = 0;
   for (int l = 0; l < num_layers; ++l) {
-    double mean = 0.0;
+    bool every = true;
+    double sum = 0.0;
     for (int i = 0; i < num_iters; ++i) {
       const double e = layer_err[(long long)l * num_iters + i];
       if (!std::isfinite(e)) return SAGE_EINVAL;
-      mean += e;
+      every = every && e > threshold;
+      sum += e;
     }
-    mean /= num_iters;
-    if (mean > threshold) layers_out[n++] = l;
+    const bool pick = rule == SAGE_SELECT_EVERY_ITERATION ? every : sum / num_iters > threshold;
+    if (pick) layers_out[n++] = l;
   }
   *n_out = n;
   return SAGE_OK;

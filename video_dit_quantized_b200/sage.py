@@ -22,6 +22,7 @@ BLK = 128
 P_SCALE = 448.0
 
 OK, EINVAL, EUNSUPPORTED, ELAUNCH, EWORKSPACE, ETIMEOUT = 0, -1, -2, -3, -4, -5
+SELECT_EVERY_ITERATION, SELECT_MEAN = 0, 1
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sage.h")
 
@@ -58,7 +59,8 @@ def _load() -> ctypes.CDLL:
         "sage_attn_quantized_ex": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
         "sage_error_scratch_bytes": (sz, [i32, i32]),
         "sage_attn_error_stats": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
-        "sage_select_full_precision_layers": (i32, [vp, i32, i32, ctypes.c_double, vp, vp]),
+        "sage_attn_rel_l2": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "sage_select_full_precision_layers": (i32, [vp, i32, i32, ctypes.c_double, i32, vp, vp]),
         "sage_quantize_blocks_2d": (i32, [vp, i32, i32, vp, vp, vp]),
         "sage_linear_w8a8": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]),
         "sage_dbg_linear_forced_timeout": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
@@ -264,22 +266,43 @@ def error_stats(a, b, stream=None):
     return stats
 
 
+def rel_l2(a, b, out=None, scratch=None, stream=None):
+    """sqrt(sum (a-b)^2 / sum b^2) over every element of two bf16 [B,H,N,d] device tensors, computed on the
+    device (sage_attn_rel_l2).  out: device fp64 tensor of one element (a view into a larger table works);
+    returned."""
+    import torch
+    B, H, N, d = _bhnd(a, "a")
+    _need(b, "b", torch.bfloat16, tuple(a.shape))
+    if out is None:
+        out = torch.empty((), dtype=torch.float64, device=a.device)
+    if scratch is None:
+        scratch = torch.empty(max(int(LIB.sage_error_scratch_bytes(B, H)), 16), dtype=torch.uint8, device=a.device)
+    _check(LIB.sage_attn_rel_l2(_dptr(a), _dptr(b), B, H, N, d, _dptr(out), _dptr(scratch),
+                                scratch.numel() * scratch.element_size(), _stream(stream)), "sage_attn_rel_l2")
+    return out
+
+
 def layer_errors(layers, stream=None):
     """Relative L2 error of the INT8/FP8 output against the BF16 output, per layer and iteration.
 
     layers: [num_layers][num_iters] of (q, k, v) device bf16 [B,H,N,d] tensors.
-    Returns a nested list [num_layers][num_iters] of sqrt(sum (a-b)^2 / sum b^2) over all heads.
+    Returns a nested list [num_layers][num_iters] of sqrt(sum (a-b)^2 / sum b^2) over all heads, each
+    formed on the device by sage_attn_rel_l2 and read back once at the end.
     """
-    out = []
-    for per_layer in layers:
-        row = []
-        for (q, k, v) in per_layer:
+    import torch
+    L = len(layers)
+    I = len(layers[0]) if L else 0
+    err = None
+    for li, per_layer in enumerate(layers):
+        if len(per_layer) != I:
+            raise ValueError("every layer needs the same number of iterations")
+        for ii, (q, k, v) in enumerate(per_layer):
+            if err is None:
+                err = torch.empty((L, I), dtype=torch.float64, device=q.device)
             oq = attn_fwd(q, k, v, MODE_INT8_FP8, stream=stream)
             ob = attn_fwd(q, k, v, MODE_BF16, stream=stream)
-            st = error_stats(oq, ob, stream=stream).sum(dim=0).cpu()
-            row.append(float((st[0] / st[1]).sqrt()))
-        out.append(row)
-    return out
+            rel_l2(oq, ob, out=err[li, ii], stream=stream)
+    return [] if err is None else err.cpu().tolist()
 
 
 def linear_layer_errors(layers, stream=None):
@@ -290,22 +313,27 @@ def linear_layer_errors(layers, stream=None):
     large run W8A16 (select_full_precision_layers on this table).
     layers: [num_layers][num_iters] of (x bf16 [M, K], wq int8 [N, K], sw fp32, bias bf16 [N] or None).
     """
-    out = []
-    for per_layer in layers:
-        row = []
-        for (x, wq, sw, bias) in per_layer:
+    import torch
+    L = len(layers)
+    I = len(layers[0]) if L else 0
+    err = None
+    for li, per_layer in enumerate(layers):
+        if len(per_layer) != I:
+            raise ValueError("every layer needs the same number of iterations")
+        for ii, (x, wq, sw, bias) in enumerate(per_layer):
+            if err is None:
+                err = torch.empty((L, I), dtype=torch.float64, device=x.device)
             xq, sx = quantize_blocks_2d(x, stream=stream)
             y8 = linear_w8a8(xq, sx, wq, sw, bias, stream=stream)
             y16 = linear_w8a16(x, wq, sw, bias, stream=stream)
             M, N = y8.shape
-            st = error_stats(y8.view(1, 1, M, N), y16.view(1, 1, M, N), stream=stream).sum(dim=0).cpu()
-            row.append(float((st[0] / st[1]).sqrt()))
-        out.append(row)
-    return out
+            rel_l2(y8.view(1, 1, M, N), y16.view(1, 1, M, N), out=err[li, ii], stream=stream)
+    return [] if err is None else err.cpu().tolist()
 
 
-def select_full_precision_layers(layer_err, threshold: float) -> list[int]:
-    """Layers whose mean error over iterations exceeds threshold; layer_err is [layers][iterations]."""
+def select_full_precision_layers(layer_err, threshold: float, rule: int = SELECT_EVERY_ITERATION) -> list[int]:
+    """Layers kept at full precision from layer_err [layers][iterations]: with SELECT_EVERY_ITERATION those
+    whose error is above threshold at every iteration, with SELECT_MEAN those whose mean error is."""
     import numpy as np
     err = np.ascontiguousarray(np.asarray(layer_err, dtype=np.float64))
     if err.ndim != 2:
@@ -314,7 +342,7 @@ def select_full_precision_layers(layer_err, threshold: float) -> list[int]:
     out = (ctypes.c_int * max(L, 1))()
     n = ctypes.c_int(0)
     _check(LIB.sage_select_full_precision_layers(err.ctypes.data_as(ctypes.c_void_p), L, I, float(threshold),
-                                                 ctypes.cast(out, ctypes.c_void_p), ctypes.byref(n)),
+                                                 int(rule), ctypes.cast(out, ctypes.c_void_p), ctypes.byref(n)),
            "sage_select_full_precision_layers")
     return [int(out[i]) for i in range(n.value)]
 
