@@ -14,7 +14,9 @@ HBM.  Metric: attention TFLOPS = 4 * B * H * N^2 * d / step time.
 `--op ulysses` times the sequence-parallel layer instead: each of N ranks holds
 N_seq / N tokens of Q, K, V for all heads; the Ulysses exchange (NCCL
 all-to-all) gives each the whole sequence for H / N heads, the INT8/FP8 path
-runs on them, and O goes back.  The total problem is fixed (strong scaling);
+runs on them straight from the receive buffers (the prepass reads the
+exchange layout, the attention epilogue writes O into the send layout of the
+return exchange), and O goes back.  The total problem is fixed (strong scaling);
 value = the full layer's attention FLOPs / max-over-ranks time.  On one GPU
 the exchange is a single-rank NCCL all-to-all (a local copy).
 
@@ -439,7 +441,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * (4 if quant else 1),
+        "gpu_launches": args.steps * (2 if quant else 1),        # prepass (one persistent kernel) + attention
         "mma_probe": {"kind": "i8" if quant else "bf16", "mac_per_clk_per_sm": probe["mac_per_clk_per_sm"],
                       "peak_at_median_sm_clock_tflops": (2 * probe["mac_per_clk_per_sm"] * probe["sms"] *
                                                          (clocks["sm_mhz"] or 0) * 1e6 / 1e12),
@@ -671,7 +673,9 @@ def run_ulysses(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
                    "parallelism": f"ulysses sp{world}", "tokens_per_rank": Nl, "heads_per_rank": w.H // world},
-        "gpu_launches": args.steps * (3 + 3 + 4 + 2),         # permutes, prepass + attention, O permutes
+        # send copies of q, k, v and the O receive copy (none at P = 1: the layouts coincide), then the
+        # fused prepass + attention (BF16: three gathers + attention)
+        "gpu_launches": args.steps * ((4 if world > 1 else 0) + (2 if mode != sage.MODE_BF16 else 4)),
         "clocks": clk.summary(),
     }), flush=True)
 
@@ -793,7 +797,7 @@ def run_stack(args, rank, world, local_rank):
                            "speedup_of_selective": ms_bf16 / ms, "clocks": clocks_bf16},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * sum(4 if m != sage.MODE_BF16 else 1 for m in modes),
+        "gpu_launches": args.steps * sum(2 if m != sage.MODE_BF16 else 1 for m in modes),
         "clocks": clocks,
     }), flush=True)
 

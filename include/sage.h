@@ -187,10 +187,14 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
  * q_dev, k_dev, v_dev, o_dev: device staging buffers bf16 [B,H,N,d] (caller-owned).
  * workspace: at least sage_workspace_bytes(1, chunk_heads, N, d, mode) bytes,
  *   reused by every chunk.
+ * The first and the last chunk take half as many heads (at least one): they
+ * are the copies nothing overlaps.
  * Runs after earlier work on `stream` and returns when the output is in
- * o_host (it synchronises); it creates and destroys two copy streams and
- * three events, and allocates no device memory.  Returns the status of the
- * call including device-side status (SAGE_ETIMEOUT).
+ * o_host (it synchronises).  Its two copy streams and three events are made
+ * on the first call on a device (and again in a new CUDA context) and kept
+ * until the process exits; calls on one device from several host threads run
+ * one after the other.  Allocates no device memory.  Returns the status of
+ * the call including device-side status (SAGE_ETIMEOUT).
  */
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H,
                        int N, int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
@@ -326,27 +330,50 @@ int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const vo
                       int M, int N, int K, void* workspace, size_t workspace_bytes, void* status, void* stream);
 
 /*
- * Layout permutations around the DeepSpeed-Ulysses all-to-all (TMAP write-up,
- * "Optimising multi-GPU parallelism": the sequence is split over P GPUs, an
- * all-to-all gives each GPU the whole sequence for H/P heads, attention runs
- * head-parallel, a second all-to-all returns O to the sequence slices).  The
- * collectives are the caller's (NCCL); these calls move rows of d bf16
- * values, Hl = H / P, N = P * Nl:
- *   SAGE_ULYSSES_SEND_QKV  src [B, Nl, H, d]      -> dst [P][B, Hl, Nl, d]
- *   SAGE_ULYSSES_RECV_QKV  src [P][B, Hl, Nl, d]  -> dst [B, Hl, N, d]
- *   SAGE_ULYSSES_SEND_O    src [B, Hl, N, d]      -> dst [P][B, Hl, Nl, d]
- *   SAGE_ULYSSES_RECV_O    src [P][B, Hl, Nl, d]  -> dst [B, Nl, H, d]
- * The [P] side has chunk_rows rows (of d values) between consecutive chunks
- * (0: dense, B*Hl*Nl) and starts base_rows rows into its buffer, so several
- * tensors can share one all-to-all buffer.  H % P == 0, d in {64, 128},
- * B, Nl, P >= 1; pointers 16-byte aligned, src and dst disjoint.
- * Asynchronous on `stream`.  Errors: SAGE_EINVAL (sizes, op, chunk_rows
- * below the dense chunk, pointers), SAGE_EUNSUPPORTED / SAGE_ELAUNCH (device).
+ * Sequence-parallel (DeepSpeed-Ulysses) attention (TMAP write-up, "Optimising
+ * multi-GPU parallelism"): each of P ranks holds Nl = N / P tokens of every
+ * head; an all-to-all gives each rank all N tokens of Hl = H / P heads,
+ * attention runs on those, and a second all-to-all returns O to the token
+ * slices.  The exchange buffers use the layout [P][B][Nl][Hl][d] (bf16):
+ * chunk r holds the sending rank's tokens for heads r*Hl .. r*Hl + Hl - 1,
+ * token-major, so that chunk p of the receive buffer holds tokens
+ * p*Nl .. p*Nl + Nl - 1 of this rank's heads.
+ *
+ * sage_attn_fwd_seqpar: O = softmax(Q K^T / sqrt(d)) V over the B x Hl heads
+ * and N = P * Nl tokens, as sage_attn_fwd, with q, k, v read from and o
+ * written to that layout (device pointers; o is the send buffer of the return
+ * exchange).  In the INT8/FP8 modes the quantization prepass reads the
+ * chunks directly and the attention epilogue writes the chunks directly, so
+ * no layout copy runs; in BF16 mode q, k, v are first gathered into the
+ * workspace.  workspace: device, 256-byte aligned, at least
+ * sage_seqpar_workspace_bytes(P, B, Nl, Hl, d, mode) bytes, status word first
+ * (sage_status).  Results are bitwise those of sage_attn_fwd on the same
+ * heads in the plain layout.  Errors as sage_attn_fwd (SAGE_EINVAL for
+ * P < 1, Nl < 1 or P * Nl above 2^30).
  */
-#define SAGE_ULYSSES_SEND_QKV 0
-#define SAGE_ULYSSES_RECV_QKV 1
-#define SAGE_ULYSSES_SEND_O 2
-#define SAGE_ULYSSES_RECV_O 3
+size_t sage_seqpar_workspace_bytes(int P, int B, int Nl, int Hl, int d, int mode);
+int sage_attn_fwd_seqpar(const void* q, const void* k, const void* v, void* o, int P, int B, int Nl, int Hl, int d,
+                         int mode, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Layout copies around the Ulysses all-to-all (rows of d bf16 values; Hl =
+ * H / P, N = P * Nl):
+ *   SAGE_ULYSSES_SEND     src [B, Nl, H, d]          -> dst [P][B][Nl][Hl][d]
+ *   SAGE_ULYSSES_RECV_O   src [P][B][Nl][Hl][d]      -> dst [B, Nl, H, d]
+ *   SAGE_ULYSSES_GATHER   src [P][B][Nl][Hl][d]      -> dst [B, Hl, N, d]
+ *   SAGE_ULYSSES_SCATTER  src [B, Hl, N, d]          -> dst [P][B][Nl][Hl][d]
+ * At P = 1 SEND and RECV_O are plain copies (the layouts coincide).  The [P]
+ * side may be strided: chunk r starts at row base_rows + r * chunk_rows
+ * (chunk_rows = 0 means dense, B*Hl*Nl; otherwise at least that), so that
+ * several tensors can share one exchange buffer.  H % P == 0, d in {64, 128},
+ * B, Nl, P >= 1; src and dst device, 16-byte aligned, disjoint.  Asynchronous
+ * on `stream`.  Errors: SAGE_EINVAL (sizes, op, chunk_rows below the dense
+ * chunk, pointers), SAGE_EUNSUPPORTED / SAGE_ELAUNCH (device).
+ */
+#define SAGE_ULYSSES_SEND 0
+#define SAGE_ULYSSES_RECV_O 1
+#define SAGE_ULYSSES_GATHER 2
+#define SAGE_ULYSSES_SCATTER 3
 int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
                          long long chunk_rows, long long base_rows, void* stream);
 

@@ -62,17 +62,28 @@ def emul_and_exact(q, k, v, rows):
 
 
 def ulysses_ref_permute(src, dst, B, Nl, H, d, P, op):
-    """The four Ulysses layout moves written with torch reshapes / permutes (dense [P] side)."""
+    """The four Ulysses layout copies written with torch reshapes / permutes (dense [P] side).
+    Exchange layout [P, B, Nl, Hl, d]: chunk r holds the sender's tokens for heads r*Hl .. r*Hl + Hl - 1."""
     Hl = H // P
-    if op == 0:      # [B, Nl, H, d] -> [P, B, Hl, Nl, d]
-        dst.copy_(src.reshape(B, Nl, P, Hl, d).permute(2, 0, 3, 1, 4))
-    elif op == 1:    # [P, B, Hl, Nl, d] -> [B, Hl, P*Nl, d]
-        dst.copy_(src.reshape(P, B, Hl, Nl, d).permute(1, 2, 0, 3, 4).reshape(B, Hl, P * Nl, d))
-    elif op == 2:    # [B, Hl, P*Nl, d] -> [P, B, Hl, Nl, d]
-        dst.copy_(src.reshape(B, Hl, P, Nl, d).permute(2, 0, 1, 3, 4))
-    else:            # [P, B, Hl, Nl, d] -> [B, Nl, H, d]
-        dst.copy_(src.reshape(P, B, Hl, Nl, d).permute(1, 3, 0, 2, 4).reshape(B, Nl, H, d))
+    if op == 0:      # send: [B, Nl, H, d] -> [P, B, Nl, Hl, d]
+        dst.copy_(src.reshape(B, Nl, P, Hl, d).permute(2, 0, 1, 3, 4))
+    elif op == 1:    # receive O: [P, B, Nl, Hl, d] -> [B, Nl, H, d]
+        dst.copy_(src.reshape(P, B, Nl, Hl, d).permute(1, 2, 0, 3, 4).reshape(B, Nl, H, d))
+    elif op == 2:    # gather: [P, B, Nl, Hl, d] -> [B, Hl, P * Nl, d]
+        dst.copy_(src.reshape(P, B, Nl, Hl, d).permute(1, 3, 0, 2, 4).reshape(B, Hl, P * Nl, d))
+    else:            # scatter: [B, Hl, P * Nl, d] -> [P, B, Nl, Hl, d]
+        dst.copy_(src.reshape(B, Hl, P, Nl, d).permute(2, 0, 3, 1, 4))
     return dst
+
+
+def attention_seqpar_ref(q, k, v, mode, o, workspace=None):
+    """attention_per_head_ref on the [P, B, Nl, Hl, d] exchange layout: gather, attend, scatter."""
+    import torch
+    P, B, Nl, Hl, d = q.shape
+    g = lambda t: t.permute(1, 3, 0, 2, 4).reshape(B, Hl, P * Nl, d)
+    out = attention_per_head_ref(g(q), g(k), g(v), mode, torch.empty((B, Hl, P * Nl, d), dtype=o.dtype))
+    o.copy_(out.reshape(B, Hl, P, Nl, d).permute(2, 0, 3, 1, 4))
+    return o
 
 
 def attention_per_head_ref(q, k, v, mode, o, workspace=None):

@@ -75,7 +75,7 @@ def _ulysses_rank(rank, world, port, result_q):
     import torch.distributed as dist
 
     import synth
-    from _util import attention_per_head_ref, ulysses_ref_permute
+    from _util import attention_per_head_ref, attention_seqpar_ref, ulysses_ref_permute
     from video_dit_quantized_b200 import sage
     from video_dit_quantized_b200.ulysses import UlyssesAttention
 
@@ -93,7 +93,7 @@ def _ulysses_rank(rank, world, port, result_q):
             return dist.all_to_all_single(out, inp, async_op=True)
 
         ua = UlyssesAttention(w.B, Nl, w.H, w.d, world, mode=sage.MODE_BF16, device="cpu",
-                              permute=ulysses_ref_permute, attention=attention_per_head_ref, a2a=a2a)
+                              permute=ulysses_ref_permute, attention=attention_seqpar_ref, a2a=a2a)
         ua.send("q", mine[0])          # q goes out before k and v exist, as a DiT block would issue it
         ua.send("k", mine[1])
         ua.send("v", mine[2])
@@ -131,13 +131,13 @@ def test_ulysses_host_checks():
     """UlyssesAttention refuses what the exchange cannot do, on the host (no GPU, no process group)."""
     import torch
 
-    from _util import attention_per_head_ref, ulysses_ref_permute
+    from _util import attention_per_head_ref, attention_seqpar_ref, ulysses_ref_permute
     from video_dit_quantized_b200 import sage
     from video_dit_quantized_b200.ulysses import UlyssesAttention
 
     with pytest.raises(ValueError):
         UlyssesAttention(1, 8, 6, 16, 4, device="cpu", permute=ulysses_ref_permute,
-                         attention=attention_per_head_ref, a2a=lambda o, i: None)      # 6 heads over 4 ranks
+                         attention=attention_seqpar_ref, a2a=lambda o, i: None)        # 6 heads over 4 ranks
     sent = []
 
     def a2a(out, inp):
@@ -146,7 +146,7 @@ def test_ulysses_host_checks():
         return None
 
     ua = UlyssesAttention(1, 8, 4, 16, 1, mode=sage.MODE_BF16, device="cpu", permute=ulysses_ref_permute,
-                          attention=attention_per_head_ref, a2a=a2a)
+                          attention=attention_seqpar_ref, a2a=a2a)
     x = torch.randn(1, 8, 4, 16).to(torch.bfloat16)
     with pytest.raises(ValueError):
         ua.send("q", torch.randn(1, 8, 2, 16).to(torch.bfloat16))                    # wrong shape
@@ -161,4 +161,4 @@ def test_ulysses_host_checks():
     ref = attention_per_head_ref(*(x.permute(0, 2, 1, 3),) * 3, sage.MODE_BF16,
                                  torch.empty(1, 4, 8, 16, dtype=torch.bfloat16))
     assert torch.equal(out.view(torch.int16), ref.permute(0, 2, 1, 3).contiguous().view(torch.int16))
-    assert sent == [(1, 1, 4, 8, 16)] * 4                                             # q, k, v, O chunks
+    assert sent == [(1, 1, 8, 4, 16)] * 4                                 # q, k, v, O: [P, B, Nl, Hl, d]

@@ -1,14 +1,17 @@
-"""Ulysses layout permutations on the GPU, and the whole exchange emulated on one GPU.
+"""Ulysses layout copies and the fused sequence-parallel attention on the GPU, and the whole
+exchange emulated on one GPU.
 
-The four row permutations of sage_ulysses_permute equal independent torch
+The four row copies of sage_ulysses_permute equal independent torch
 reshape/permute references bit for bit, dense and with a strided [P] side.
-With P ranks emulated on one device (the all-to-all done by slicing the P
-send buffers), the sequence-parallel path -- permute, exchange, quantized or
-BF16 attention on the local heads, permute back, exchange, permute -- gives
-the same bits as one attention call over all heads: attention has no
-cross-head term and the kernels treat every (b, h) alike.  The pattern is the
-DeepSpeed-Ulysses sequence parallelism of the TMAP write-up ("Optimising
-multi-GPU parallelism").
+sage_attn_fwd_seqpar, which reads q, k, v from the exchange layout
+[P][B][Nl][Hl][d] and writes O into it (the quantization prepass walks the
+chunks, the attention epilogue scatters its rows), gives the same bits as
+sage_attn_fwd on the gathered heads, in every mode, with ragged chunks.  With
+P ranks emulated on one device (the all-to-all done by slicing the P send
+buffers), the sequence-parallel path gives the same bits as one attention
+call over all heads: attention has no cross-head term and the kernels treat
+every (b, h) alike.  The pattern is the DeepSpeed-Ulysses sequence
+parallelism of the TMAP write-up ("Optimising multi-GPU parallelism").
 """
 import numpy as np
 import pytest
@@ -31,8 +34,8 @@ def test_permutes_match_reference(B, Nl, H, d, P, cuda_dev):
     from video_dit_quantized_b200 import sage
     g = torch.Generator(device="cpu").manual_seed(B * 1000 + Nl + H + P)
     Hl, N = H // P, P * Nl
-    shapes_in = {0: (B, Nl, H, d), 1: (P, B, Hl, Nl, d), 2: (B, Hl, N, d), 3: (P, B, Hl, Nl, d)}
-    shapes_out = {0: (P, B, Hl, Nl, d), 1: (B, Hl, N, d), 2: (P, B, Hl, Nl, d), 3: (B, Nl, H, d)}
+    shapes_in = {0: (B, Nl, H, d), 1: (P, B, Nl, Hl, d), 2: (P, B, Nl, Hl, d), 3: (B, Hl, N, d)}
+    shapes_out = {0: (P, B, Nl, Hl, d), 1: (B, Nl, H, d), 2: (B, Hl, N, d), 3: (P, B, Nl, Hl, d)}
     for op in range(4):
         src = torch.randn(shapes_in[op], generator=g).to(torch.bfloat16).to(cuda_dev)
         got = torch.empty(shapes_out[op], dtype=torch.bfloat16, device=cuda_dev)
@@ -40,23 +43,47 @@ def test_permutes_match_reference(B, Nl, H, d, P, cuda_dev):
         want = ulysses_ref_permute(src, torch.empty_like(got), B, Nl, H, d, P, op)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int16), want.view(torch.int16)), op
-    # strided [P] side: q, k, v interleaved as [P][3][B, Hl, Nl, d]
+    # strided [P] side: q, k, v interleaved as [P][3][B][Nl][Hl][d]
     dense = B * Hl * Nl
     x = torch.randn((3, B, Nl, H, d), generator=g).to(torch.bfloat16).to(cuda_dev)
-    buf = torch.zeros((P, 3, B, Hl, Nl, d), dtype=torch.bfloat16, device=cuda_dev)
+    buf = torch.zeros((P, 3, B, Nl, Hl, d), dtype=torch.bfloat16, device=cuda_dev)
     for t in range(3):
-        sage.ulysses_permute(x[t], buf, B, Nl, H, d, P, 0, chunk_rows=3 * dense, base_rows=t * dense)
+        sage.ulysses_permute(x[t], buf, B, Nl, H, d, P, sage.ULYSSES_SEND, chunk_rows=3 * dense, base_rows=t * dense)
     back = torch.empty_like(x)
     for t in range(3):
-        want = ulysses_ref_permute(x[t], torch.empty((P, B, Hl, Nl, d), dtype=torch.bfloat16, device=cuda_dev),
+        want = ulysses_ref_permute(x[t], torch.empty((P, B, Nl, Hl, d), dtype=torch.bfloat16, device=cuda_dev),
                                    B, Nl, H, d, P, 0)
         assert torch.equal(buf[:, t].view(torch.int16), want.view(torch.int16))
-        sage.ulysses_permute(buf, back[t], B, Nl, H, d, P, 3, chunk_rows=3 * dense, base_rows=t * dense)
+        sage.ulysses_permute(buf, back[t], B, Nl, H, d, P, sage.ULYSSES_RECV_O, chunk_rows=3 * dense,
+                             base_rows=t * dense)
     torch.cuda.synchronize()
-    assert torch.equal(back.view(torch.int16), x.view(torch.int16))       # op 3 inverts op 0
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))       # RECV_O inverts SEND
 
 
-@pytest.mark.parametrize("mode_name,P", [("int8_fp8", 4), ("bf16", 2), ("int8_fp8", 8)])
+@pytest.mark.parametrize("mode_name,P,Nl,Hl,d", [("int8_fp8", 8, 1181, 2, 128), ("int8_fp8", 3, 333, 3, 64),
+                                                 ("int8_fp8_qtoken", 4, 257, 2, 128), ("bf16", 8, 1181, 2, 128),
+                                                 ("bf16", 1, 640, 4, 64), ("int8_fp8", 1, 1000, 3, 128)])
+def test_seqpar_equals_plain_attention(mode_name, P, Nl, Hl, d, cuda_dev):
+    """The fused chunk-layout call gives bitwise the plain call's output on the gathered heads."""
+    import torch
+    from video_dit_quantized_b200 import sage
+    mode = {"int8_fp8": sage.MODE_INT8_FP8, "int8_fp8_qtoken": sage.MODE_INT8_FP8_QTOKEN,
+            "bf16": sage.MODE_BF16}[mode_name]
+    B, N, H = 1, P * Nl, P * Hl
+    w = synth.Workload("sp", B, Hl, N, d, seed=P * 10 + Hl, outlier_frac=0.01)
+    q, k, v = (_bf16(a, cuda_dev) for a in synth.qkv_numpy(w))             # plain [B, Hl, N, d]
+    scat = lambda t: ulysses_ref_permute(t, torch.empty((P, B, Nl, Hl, d), dtype=t.dtype, device=cuda_dev),
+                                         B, Nl, H, d, P, 3)
+    qc, kc, vc = scat(q), scat(k), scat(v)
+    ws = sage.alloc_seqpar_workspace(P, B, Nl, Hl, d, mode, cuda_dev)
+    oc = sage.attn_fwd_seqpar(qc, kc, vc, mode, P=P, workspace=ws)
+    assert sage.status(ws) == sage.OK
+    ref = sage.attn_fwd(q, k, v, mode)
+    torch.cuda.synchronize()
+    assert torch.equal(oc.view(torch.int16), scat(ref).view(torch.int16))
+
+
+@pytest.mark.parametrize("mode_name,P", [("int8_fp8", 4), ("bf16", 2), ("int8_fp8", 8), ("int8_fp8", 1)])
 def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
     import torch
     from video_dit_quantized_b200 import sage
@@ -94,7 +121,7 @@ def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
 
     for r, ua in enumerate(ranks):
         for t, x in zip("qkv", seq):
-            ua.send(t, x[:, r * Nl:(r + 1) * Nl])
+            ua.send(t, x[:, r * Nl:(r + 1) * Nl].contiguous())
     exchange()
     for ua in ranks:
         ua.attend_local()

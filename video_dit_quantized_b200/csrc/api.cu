@@ -16,6 +16,28 @@
 
 namespace sage {
 
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -32,6 +54,46 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Side streams and events of sage_attn_fwd_host, made on first use per device
+// (and again in a new CUDA context) and kept for the life of the process.  A
+// call holds its device's lock, so host calls on one device run one after
+// the other.
+struct HostPipe {
+  std::mutex mu;
+  unsigned long long ctx = 0;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_done = nullptr;
+};
+constexpr int kMaxHostDevices = 64;
+HostPipe g_pipes[kMaxHostDevices];
+
+// Makes the pipe's handles in the current context if they are missing or
+// belong to an earlier one.  Called with p.mu held.
+bool pipe_ready(HostPipe& p) {
+  const unsigned long long ctx = current_context_id();
+  if (p.s_in && ctx != 0 && ctx == p.ctx) return true;
+  // handles of an earlier context are gone with it
+  p.s_in = p.s_out = nullptr;
+  p.ev_start = p.ev_in = p.ev_done = nullptr;
+  bool ok = cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.ev_start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.ev_in, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.ev_done, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    if (p.s_in) cudaStreamDestroy(p.s_in);
+    if (p.s_out) cudaStreamDestroy(p.s_out);
+    if (p.ev_start) cudaEventDestroy(p.ev_start);
+    if (p.ev_in) cudaEventDestroy(p.ev_in);
+    if (p.ev_done) cudaEventDestroy(p.ev_done);
+    p.s_in = p.s_out = nullptr;
+    p.ev_start = p.ev_in = p.ev_done = nullptr;
+    return false;
+  }
+  p.ctx = ctx;
+  return true;
+}
 
 // Workspace layout of the INT8/FP8 mode; every region 256-byte aligned.
 struct Layout {
@@ -178,6 +240,31 @@ int sage_attn_quantized_ex(const int8_t* q_i8, const float* q_scale, const int8_
                                         static_cast<cudaStream_t>(stream), q_granularity == 1));
 }
 
+namespace sage {
+namespace {
+// The INT8/FP8 path (prepass + attention) over a workspace laid out by layout();
+// q, k, v rows found through in_map, output rows written through o_map.
+int run_quantized(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, bool qtok,
+                  char* ws, cudaStream_t st, RowMap in_map, RowMap o_map) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  const Layout L = layout(B, H, N, d, qtok);
+  auto q_i8 = reinterpret_cast<int8_t*>(ws + L.q_i8);
+  auto k_i8 = reinterpret_cast<int8_t*>(ws + L.k_i8);
+  auto v_f8t = reinterpret_cast<uint8_t*>(ws + L.v_f8t);
+  auto q_scale = reinterpret_cast<float*>(ws + L.q_scale);
+  auto k_scale = reinterpret_cast<float*>(ws + L.k_scale);
+  auto k_mean = reinterpret_cast<float*>(ws + L.k_mean);
+  auto v_scale = reinterpret_cast<float*>(ws + L.v_scale);
+  const PrepassScratch s = prepass_scratch_carve(ws + L.scratch, B * H, N, d);
+  cudaError_t e =
+      launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st, qtok, in_map);
+  if (e != cudaSuccess) return launch_status(e);
+  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
+                                        kDefaultTimeoutCycles, 0, st, qtok, o_map));
+}
+}  // namespace
+}  // namespace sage
+
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int mode,
                   void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_shape(B, H, N, d);
@@ -194,21 +281,47 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   if (mode == SAGE_MODE_BF16)
     return launch_status(launch_attn_bf16(q, k, v, o, B * H, N, d, status, kDefaultTimeoutCycles, st));
-  const bool qtok = mode == SAGE_MODE_INT8_FP8_QTOKEN;
-  const Layout L = layout(B, H, N, d, qtok);
-  auto q_i8 = reinterpret_cast<int8_t*>(ws + L.q_i8);
-  auto k_i8 = reinterpret_cast<int8_t*>(ws + L.k_i8);
-  auto v_f8t = reinterpret_cast<uint8_t*>(ws + L.v_f8t);
-  auto q_scale = reinterpret_cast<float*>(ws + L.q_scale);
-  auto k_scale = reinterpret_cast<float*>(ws + L.k_scale);
-  auto k_mean = reinterpret_cast<float*>(ws + L.k_mean);
-  auto v_scale = reinterpret_cast<float*>(ws + L.v_scale);
-  const PrepassScratch s = prepass_scratch_carve(ws + L.scratch, B * H, N, d);
-  cudaError_t e =
-      launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st, qtok);
-  if (e != cudaSuccess) return launch_status(e);
-  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
-                                        kDefaultTimeoutCycles, 0, st, qtok));
+  const RowMap plain{0, 0, 0, 0};
+  return run_quantized(q, k, v, o, B, H, N, d, mode == SAGE_MODE_INT8_FP8_QTOKEN, ws, st, plain, plain);
+}
+
+size_t sage_seqpar_workspace_bytes(int P, int B, int Nl, int Hl, int d, int mode) {
+  if (P < 1 || Nl < 1 || (long long)P * Nl > (1LL << 30)) return 0;
+  const int N = P * Nl;
+  if (check_shape(B, Hl, N, d) != SAGE_OK) return 0;
+  if (mode == SAGE_MODE_BF16) return 256 + 3 * align_up((size_t)B * Hl * N * d * 2, 256);
+  return sage_workspace_bytes(B, Hl, N, d, mode);
+}
+
+int sage_attn_fwd_seqpar(const void* q, const void* k, const void* v, void* o, int P, int B, int Nl, int Hl, int d,
+                         int mode, void* workspace, size_t workspace_bytes, void* stream) {
+  if (P < 1 || Nl < 1 || (long long)P * Nl > (1LL << 30)) return SAGE_EINVAL;
+  const int N = P * Nl;
+  int rc = check_shape(B, Hl, N, d);
+  if (rc != SAGE_OK) return rc;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_INT8_FP8_QTOKEN) return SAGE_EINVAL;
+  const void* ptrs[] = {q, k, v, o, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SAGE_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_EINVAL;
+  if (workspace_bytes < sage_seqpar_workspace_bytes(P, B, Nl, Hl, d, mode)) return SAGE_EWORKSPACE;
+  if ((rc = check_device()) != SAGE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const RowMap chunks{P, B, Nl, Hl};
+  if (mode != SAGE_MODE_BF16)
+    return run_quantized(q, k, v, o, B, Hl, N, d, mode == SAGE_MODE_INT8_FP8_QTOKEN, ws, st, chunks, chunks);
+  // BF16: the kernel's TMA tiles need the plain layout, so q, k, v are gathered first; O is
+  // written straight into the chunk layout
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  const size_t region = align_up((size_t)B * Hl * N * d * 2, 256);
+  char* g[3] = {ws + 256, ws + 256 + region, ws + 256 + 2 * region};
+  const void* src[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    const cudaError_t e = launch_ulysses_permute(src[i], g[i], B, Nl, P * Hl, d, P, SAGE_ULYSSES_GATHER, 0, 0, st);
+    if (e != cudaSuccess) return launch_status(e);
+  }
+  return launch_status(launch_attn_bf16(g[0], g[1], g[2], o, B * Hl, N, d, status, kDefaultTimeoutCycles, st, chunks));
 }
 
 int sage_host_chunk_heads(int B, int H, int N, int d) {
@@ -244,24 +357,14 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   if (workspace_bytes < sage_workspace_bytes(1, chunk_heads, N, d, mode)) return SAGE_EWORKSPACE;
   if ((rc = check_device()) != SAGE_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess) return SAGE_ELAUNCH;
-  if (cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess) {
-    cudaStreamDestroy(s_in);
-    return SAGE_ELAUNCH;
-  }
-  // inputs of chunk i land (s_in) -> its attention runs (stream) -> its output leaves (s_out)
-  cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_done = nullptr;
-  if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) != cudaSuccess) {
-    if (ev_start) cudaEventDestroy(ev_start);
-    if (ev_in) cudaEventDestroy(ev_in);
-    if (ev_done) cudaEventDestroy(ev_done);
-    cudaStreamDestroy(s_in);
-    cudaStreamDestroy(s_out);
-    return SAGE_ELAUNCH;
-  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxHostDevices) return SAGE_ELAUNCH;
+  HostPipe& pipe = g_pipes[dev];
+  std::lock_guard<std::mutex> lock(pipe.mu);
+  if (!pipe_ready(pipe)) return SAGE_ELAUNCH;
+  cudaStream_t s_in = pipe.s_in, s_out = pipe.s_out;
+  cudaEvent_t ev_start = pipe.ev_start, ev_in = pipe.ev_in, ev_done = pipe.ev_done;
+  // inputs of chunk i land (s_in) -> its attention runs (stream) -> its output leaves (s_out);
   // copies may not start before earlier work on the caller's stream
   cudaEventRecord(ev_start, st);
   cudaStreamWaitEvent(s_in, ev_start, 0);
@@ -274,9 +377,15 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   char* kd = static_cast<char*>(k_dev);
   char* vd = static_cast<char*>(v_dev);
   char* od = static_cast<char*>(o_dev);
+  // The first and the last chunk take half as many heads: the first upload and
+  // the last download are the parts of the pipeline nothing overlaps.
+  const int half = std::max(1, chunk_heads / 2);
+  const int first = std::min(half, BH);
+  const int last = std::min(half, BH - first);
   rc = SAGE_OK;
-  for (int i = 0; i < n_chunks && rc == SAGE_OK; ++i) {
-    const int h0 = i * chunk_heads, hc = std::min(chunk_heads, BH - h0);
+  for (int h0 = 0; h0 < BH && rc == SAGE_OK;) {
+    int hc = h0 == 0 ? first : std::min(chunk_heads, BH - last - h0);
+    if (hc <= 0) hc = BH - h0;                       // the last chunk
     const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hc * head_bytes;
     if (cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
         cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
@@ -290,16 +399,12 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
     if (cudaEventRecord(ev_done, st) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
         cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
       rc = SAGE_ELAUNCH;
+    h0 += hc;
   }
   // the caller's stream resumes after the last output copy
   cudaEventRecord(ev_done, s_out);
   cudaStreamWaitEvent(st, ev_done, 0);
   if (cudaStreamSynchronize(s_out) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) rc = SAGE_ELAUNCH;
-  cudaEventDestroy(ev_start);
-  cudaEventDestroy(ev_in);
-  cudaEventDestroy(ev_done);
-  cudaStreamDestroy(s_in);
-  cudaStreamDestroy(s_out);
   if (rc != SAGE_OK) return rc;
   return sage_status(workspace, stream);
 }
@@ -427,7 +532,7 @@ int sage_linear_w8a16(const void* x, const int8_t* wq, const float* sw, const vo
 int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
                          long long chunk_rows, long long base_rows, void* stream) {
   if (B < 1 || Nl < 1 || H < 1 || P < 1 || H % P != 0 || (d != 64 && d != 128)) return SAGE_EINVAL;
-  if (op < SAGE_ULYSSES_SEND_QKV || op > SAGE_ULYSSES_RECV_O || chunk_rows < 0 || base_rows < 0) return SAGE_EINVAL;
+  if (op < SAGE_ULYSSES_SEND || op > SAGE_ULYSSES_SCATTER || chunk_rows < 0 || base_rows < 0) return SAGE_EINVAL;
   if (!src || !dst || !aligned16(src) || !aligned16(dst) || src == dst) return SAGE_EINVAL;
   const long long rows = (long long)B * Nl * H;
   const long long dense = (long long)B * (H / P) * Nl;

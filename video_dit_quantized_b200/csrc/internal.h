@@ -16,6 +16,20 @@ constexpr uint32_t kStatusTimeout = 1u;
 inline int num_tiles(int N) { return (N + kTile - 1) / kTile; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Where token n of head bh sits, in rows of d values.  P == 0: the plain
+// [BH, N, d] layout, row bh * N + n.  P >= 1: the sequence-parallel chunk
+// layout [P][B][Nl][Hl][d] (chunk p holds tokens p*Nl .. p*Nl + Nl - 1 of the
+// B x Hl heads, token-major), row ((p*B + b)*Nl + n % Nl)*Hl + h for
+// bh = b*Hl + h, p = n / Nl.
+struct RowMap {
+  int P, B, Nl, Hl;
+  __host__ __device__ long long row(int bh, int n, int N) const {
+    if (P == 0) return (long long)bh * N + n;
+    const int b = bh / Hl, h = bh - b * Hl, p = n / Nl, nl = n - p * Nl;
+    return (((long long)p * B + b) * Nl + nl) * Hl + h;
+  }
+};
+
 // Prepass scratch: per (bh, key block, channel) fp64 partial sums, fp32
 // block min / max of K and block absmax of V; per (bh, channel) V absmax.
 struct PrepassScratch {
@@ -29,20 +43,22 @@ size_t prepass_scratch_bytes(int BH, int N, int d);
 PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d);
 
 // q_per_token: q_scale is [BH, Npad] (one scale per token) instead of [BH, nT].
+// in_map: where token n of head bh sits in q, k and v.
 cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
                            float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
                            float* v_scale, const PrepassScratch& scratch, cudaStream_t stream,
-                           bool q_per_token = false);
+                           bool q_per_token = false, RowMap in_map = RowMap{0, 0, 0, 0});
 
 // Quantized attention (INT8 QK^T, FP8 PV).  status: device uint32 word.
 cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
                              const uint8_t* v_f8t, const float* v_scale, void* o, int BH, int N, int d,
                              uint32_t* status, long long timeout_cycles, int dbg_flags, cudaStream_t stream,
-                             bool q_per_token = false);
+                             bool q_per_token = false, RowMap o_map = RowMap{0, 0, 0, 0});
 
 // BF16 attention.
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, void* o, int BH, int N, int d,
-                             uint32_t* status, long long timeout_cycles, cudaStream_t stream);
+                             uint32_t* status, long long timeout_cycles, cudaStream_t stream,
+                             RowMap o_map = RowMap{0, 0, 0, 0});
 
 // 8-bit linear layers with 128 x 128 block scales.
 cudaError_t launch_quant_blocks_2d(const void* x, int R, int K, int8_t* codes, float* scales, cudaStream_t stream);
@@ -75,6 +91,10 @@ bool encode_tmap_2d(void* map, CUtensorMapDataType dtype, const void* base, uint
 bool encode_tmap_3d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
                     uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
                     uint32_t box2, CUtensorMapSwizzle swizzle);
+
+// Unique id of the current CUDA context (0 if it cannot be read); a new id
+// after cudaDeviceReset tells cached per-device handles to be made again.
+unsigned long long current_context_id();
 
 // Default wait limit of the bounded device waits, in SM clocks (~1-2 s).
 constexpr long long kDefaultTimeoutCycles = 2000000000LL;

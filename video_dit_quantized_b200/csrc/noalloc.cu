@@ -16,8 +16,6 @@
 // with the unique id of the CUDA context it belongs to.  A call in another
 // context (after cudaDeviceReset, or a destroyed and re-created primary
 // context, which reloads the module at a new address) looks it up again.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -38,30 +36,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 unsigned long long g_scratch_ctx[kMaxDevices] = {};
-
-// Unique id of the current CUDA context (through the driver entry points, so
-// the library needs no libcuda link); 0 if it cannot be read.
-unsigned long long current_context_id() {
-  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
-    return 0;
-  return id;
-}
 
 // Device address of g_prepass_scratch on the current device, looked up with
 // that device current the first time it is needed in the current context.

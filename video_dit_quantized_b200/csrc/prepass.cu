@@ -3,7 +3,8 @@
 // SageAttention operator; zero-channel fix under "operator details").
 //
 // Three HBM-bound kernels, one CTA per (128-token block, head) where a block
-// is involved:
+// is involved (the inputs are read through a RowMap: the plain [B,H,N,d]
+// layout, or the sequence-parallel exchange layout [P][B][Nl][Hl][d]):
 //   stats     : Q block -> absmax -> INT8 codes + q_scale (single pass);
 //               K block -> per-channel fp64 partial sums (ascending tokens),
 //               fp32 min / max;  V block -> per-channel absmax.
@@ -62,12 +63,13 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 
 // grid (nK, BH).  TOKQ: Q gets one scale per token (q_scale [BH, Npad]) instead
 // of one per 128-token block (q_scale [BH, nK]).
-template <int D, bool TOKQ>
+template <int D, bool TOKQ, bool CHUNKED>
 __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __restrict__ q,
                                                                  const uint4* __restrict__ k,
                                                                  const uint4* __restrict__ v, int N, int Npad,
                                                                  int8_t* __restrict__ q_i8,
-                                                                 float* __restrict__ q_scale, PrepassScratch scr) {
+                                                                 float* __restrict__ q_scale, PrepassScratch scr,
+                                                                 RowMap in_map) {
   constexpr int V8 = D / 8;                        // uint4 per token row
   constexpr int PER_T = kTile * V8 / kThreads;     // uint4 per thread per block
   static_assert(kThreads % V8 == 0, "a thread must always see the same 8 channels");
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
   const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
   const int n0 = kb * kTile;
   const int nr = min(kTile, N - n0);
-  const size_t in_base = ((size_t)bh * N + n0) * V8;  // in uint4
+  const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
 
   if (threadIdx.x < D) vamax_s[threadIdx.x] = 0;
 
@@ -92,10 +94,11 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
     const int row = e / V8;
     qv[i] = make_uint4(0, 0, 0, 0);
     if (row < nr) {
-      qv[i] = q[in_base + e];
-      ks[e] = k[in_base + e];
+      const size_t at = CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e;
+      qv[i] = q[at];
+      ks[e] = k[at];
       float y[8];
-      unpack8(v[in_base + e], y);
+      unpack8(v[at], y);
 #pragma unroll
       for (int u = 0; u < 8; ++u) va[u] = fmaxf(va[u], fabsf(y[u]));
     }
@@ -185,13 +188,14 @@ __global__ void prepass_finalize_kernel(int N, int nK, PrepassScratch scr, float
 }
 
 // grid (nK, BH)
-template <int D>
+template <int D, bool CHUNKED>
 __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4* __restrict__ k,
                                                                     const uint4* __restrict__ v, int N, int Npad,
                                                                     const float* __restrict__ k_mean,
                                                                     int8_t* __restrict__ k_i8,
                                                                     float* __restrict__ k_scale,
-                                                                    uint8_t* __restrict__ v_f8t, PrepassScratch scr) {
+                                                                    uint8_t* __restrict__ v_f8t, PrepassScratch scr,
+                                                                    RowMap in_map) {
   constexpr int V8 = D / 8;
   constexpr int PER_T = kTile * V8 / kThreads;
   __shared__ float mean_s[D];
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
   const int n0 = kb * kTile;
   const int nr = min(kTile, N - n0);
-  const size_t in_base = ((size_t)bh * N + n0) * V8;
+  const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
   const size_t pidx = ((size_t)bh * nK + kb) * D;
 
   // k_scale of this block from the partial min / max: fp32 subtraction is
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
     int c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (row < nr && kinv > 0.f) {
       float x[8];
-      unpack8(k[in_base + e], x);
+      unpack8(k[CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e], x);
 #pragma unroll
       for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
     }
@@ -241,7 +245,8 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   for (int i = 0; i < PER_T; ++i) {
     const int e = threadIdx.x + i * kThreads;
     const int row = e / V8;
-    vs[e] = row < nr ? v[in_base + e] : make_uint4(0, 0, 0, 0);
+    vs[e] = row < nr ? v[CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e]
+                     : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(vs);
@@ -271,21 +276,29 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
 template <int D>
 cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH, int N, int8_t* q_i8,
                              float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
-                             float* v_scale, const PrepassScratch& scr, bool q_per_token, cudaStream_t stream) {
+                             float* v_scale, const PrepassScratch& scr, bool q_per_token, cudaStream_t stream,
+                             RowMap in_map) {
   const int nK = num_tiles(N), Npad = nK * kTile;
   dim3 grid(nK, BH);
-  if (q_per_token)
-    prepass_stats_kernel<D, true><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
-        q_scale, scr);
+  const uint4* q4 = static_cast<const uint4*>(q);
+  const uint4* k4 = static_cast<const uint4*>(k);
+  const uint4* v4 = static_cast<const uint4*>(v);
+  const bool chunked = in_map.P != 0;
+  if (q_per_token && chunked)
+    prepass_stats_kernel<D, true, true><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
+  else if (q_per_token)
+    prepass_stats_kernel<D, true, false><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
+  else if (chunked)
+    prepass_stats_kernel<D, false, true><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
   else
-    prepass_stats_kernel<D, false><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), N, Npad, q_i8,
-        q_scale, scr);
+    prepass_stats_kernel<D, false, false><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
   prepass_finalize_kernel<D><<<BH, D, 0, stream>>>(N, nK, scr, k_mean, v_scale);
-  prepass_quant_kv_kernel<D><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(k),
-                                                            static_cast<const uint4*>(v), N, Npad, k_mean, k_i8,
-                                                            k_scale, v_f8t, scr);
+  if (chunked)
+    prepass_quant_kv_kernel<D, true><<<grid, kThreads, 0, stream>>>(k4, v4, N, Npad, k_mean, k_i8, k_scale, v_f8t, scr,
+                                                                    in_map);
+  else
+    prepass_quant_kv_kernel<D, false><<<grid, kThreads, 0, stream>>>(k4, v4, N, Npad, k_mean, k_i8, k_scale, v_f8t, scr,
+                                                                     in_map);
   return cudaGetLastError();
 }
 
@@ -314,13 +327,14 @@ PrepassScratch prepass_scratch_carve(void* base, int BH, int N, int d) {
 
 cudaError_t launch_prepass(const void* q, const void* k, const void* v, int BH, int N, int d, int8_t* q_i8,
                            float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, uint8_t* v_f8t,
-                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream, bool q_per_token) {
+                           float* v_scale, const PrepassScratch& scratch, cudaStream_t stream, bool q_per_token,
+                           RowMap in_map) {
   if (d == 128)
     return launch_prepass_d<128>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
-                                 q_per_token, stream);
+                                 q_per_token, stream, in_map);
   if (d == 64)
     return launch_prepass_d<64>(q, k, v, BH, N, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, scratch,
-                                q_per_token, stream);
+                                q_per_token, stream, in_map);
   return cudaErrorInvalidValue;
 }
 

@@ -153,6 +153,16 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Placed right after tmem_wait_ld(): makes the compiler treat r as produced
+// here (no instruction is emitted), so no use of the loaded registers can be
+// moved above the wait.  Lets one wait cover several loads.
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- MMA -------
@@ -291,6 +301,39 @@ __device__ __forceinline__ float2 fmul2(float2 a, float b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b, b)));
   return f2_unpack(d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)));
+  return f2_unpack(d);
+}
+// a * b + c, lane by lane, each rounded once
+__device__ __forceinline__ float2 ffma2v(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)), "l"(f2_pack(c.x, c.y)));
+  return f2_unpack(d);
+}
+// 2^x for a pair of floats on the FMA pipe (Cody-Waite style split):
+//   x = j + f with j = rne(x) (read off the sum x + 1.5 * 2^23) and f in
+//   [-1/2, 1/2]; 2^f by the degree-3 polynomial of least maximum relative
+//   error on that interval (Remez exchange; 7.5e-5); 2^j added into the
+//   exponent field.  x is first raised to -125 so that 2^j stays a normal
+//   number: results below 2^-125 come out as about 2^-125 instead of smaller,
+//   which is below what any caller here keeps (P * 448 < 2^-10 rounds to e4m3
+//   zero).  x must be below 128.
+constexpr float kExp2C0 = 0.9999280735394012f, kExp2C1 = 0.6932609854606553f, kExp2C2 = 0.2426111221932161f,
+                kExp2C3 = 0.05517166905792616f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 M = make_float2(12582912.f, 12582912.f);
+  const float2 t = fadd2(x, M);
+  const float2 f = fsub2(x, fsub2(t, M));
+  float2 p = ffma2v(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  p = ffma2v(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2v(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 // Packs four floats (element 0 in the low byte) as e4m3, RNE, saturating to +-448.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {

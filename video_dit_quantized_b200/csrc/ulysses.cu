@@ -1,21 +1,24 @@
-// ulysses.cu -- layout permutations around the DeepSpeed-Ulysses all-to-all.
+// ulysses.cu -- layout copies around the DeepSpeed-Ulysses all-to-all.
 //
 // TMAP write-up, "Optimising multi-GPU parallelism" (DeepSpeed-Ulysses
 // sequence parallelism): each GPU holds a 1/P slice of the sequence for all H
 // heads; an all-to-all hands every GPU the whole sequence for H/P heads,
 // attention runs per head, and a second all-to-all returns the output to the
-// sequence slices.  The collectives
-// themselves are NCCL's; these kernels only move rows of d contiguous bf16
-// values between the four layouts (Hl = H / P, N = P * Nl):
+// sequence slices.  The collectives themselves are NCCL's; these kernels only
+// move rows of d contiguous bf16 values between the layouts (Hl = H / P,
+// N = P * Nl).  The exchange buffers are [P][B][Nl][Hl][d]: chunk r holds the
+// sending rank's tokens for heads r*Hl .. r*Hl + Hl - 1, token-major, so one
+// token's heads of one chunk are Hl consecutive rows.
 //
-//   op 0  send Q/K/V:  x [B, Nl, H, d]          -> s [P][B, Hl, Nl, d]
-//   op 1  recv Q/K/V:  r [P][B, Hl, Nl, d]      -> y [B, Hl, N, d]  (the attention layout)
-//   op 2  send O:      o [B, Hl, N, d]          -> s [P][B, Hl, Nl, d]
-//   op 3  recv O:      r [P][B, Hl, Nl, d]      -> y [B, Nl, H, d]
+//   op 0  send:     x [B, Nl, H, d]          -> s [P][B][Nl][Hl][d]
+//   op 1  recv O:   r [P][B][Nl][Hl][d]      -> y [B, Nl, H, d]
+//   op 2  gather:   r [P][B][Nl][Hl][d]      -> y [B, Hl, N, d]  (the plain attention layout)
+//   op 3  scatter:  y [B, Hl, N, d]          -> s [P][B][Nl][Hl][d]
 //
-// The [P] side may be strided (chunk_rows rows between consecutive chunks,
-// first chunk at row base_rows) so that Q, K and V share one send buffer
-// [P][3][B, Hl, Nl, d] and one all-to-all.
+// sage_attn_fwd_seqpar reads and writes the [P] layout directly in INT8/FP8
+// mode; ops 2 and 3 serve the BF16 mode and tests.  The [P] side may be
+// strided (chunk_rows rows between consecutive chunks, first chunk at row
+// base_rows), so that several tensors can share one exchange buffer.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -31,35 +34,35 @@ struct UlyGeom {
   long long chunk_rows, base_rows;  // of the [P] side
 };
 
-// Source row of destination row i.
+// Row of the [P] side holding (chunk r, b, token n of the chunk, head hl).
+__device__ __forceinline__ long long p_row(const UlyGeom& g, long long r, long long b, long long n, long long hl) {
+  return g.base_rows + r * g.chunk_rows + (b * g.Nl + n) * g.Hl + hl;
+}
+
+// Source row of destination row i (i enumerates the destination densely).
 __device__ __forceinline__ long long src_row(long long i, int op, const UlyGeom& g) {
-  if (op == 0) {  // dst (r, b, hl, n) in the [P] buffer <- x (b, n, r*Hl + hl)
-    const long long inner = g.B * g.Hl * g.Nl;
+  if (op == 0 || op == 3) {  // dst (r, b, n, hl) in the [P] buffer
+    const long long inner = g.B * g.Nl * g.Hl;
     const long long r = i / inner, q = i - r * inner;
-    const long long b = q / (g.Hl * g.Nl), hl = (q / g.Nl) % g.Hl, n = q % g.Nl;
-    return (b * g.Nl + n) * g.H + r * g.Hl + hl;
+    const long long b = q / (g.Nl * g.Hl), n = (q / g.Hl) % g.Nl, hl = q % g.Hl;
+    if (op == 0) return (b * g.Nl + n) * g.H + r * g.Hl + hl;     // x (b, n, r*Hl + hl)
+    return (b * g.Hl + hl) * g.N + r * g.Nl + n;                  // y (b, hl, r*Nl + n)
   }
-  if (op == 1) {  // dst (b, hl, tok) <- [P] buffer (tok / Nl, b, hl, tok % Nl)
-    const long long b = i / (g.Hl * g.N), hl = (i / g.N) % g.Hl, tok = i % g.N;
-    const long long r = tok / g.Nl, n = tok - r * g.Nl;
-    return g.base_rows + r * g.chunk_rows + (b * g.Hl + hl) * g.Nl + n;
+  if (op == 1) {  // dst (b, n, h) <- [P] buffer (h / Hl, b, n, h % Hl)
+    const long long b = i / (g.Nl * g.H), n = (i / g.H) % g.Nl, h = i % g.H;
+    const long long r = h / g.Hl;
+    return p_row(g, r, b, n, h - r * g.Hl);
   }
-  if (op == 2) {  // dst (r, b, hl, n) in the [P] buffer <- o (b, hl, r*Nl + n)
-    const long long inner = g.B * g.Hl * g.Nl;
-    const long long r = i / inner, q = i - r * inner;
-    const long long b = q / (g.Hl * g.Nl), hl = (q / g.Nl) % g.Hl, n = q % g.Nl;
-    return (b * g.Hl + hl) * g.N + r * g.Nl + n;
-  }
-  // op 3: dst (b, n, h) <- [P] buffer (h / Hl, b, h % Hl, n)
-  const long long b = i / (g.Nl * g.H), n = (i / g.H) % g.Nl, h = i % g.H;
-  const long long r = h / g.Hl, hl = h - r * g.Hl;
-  return g.base_rows + r * g.chunk_rows + (b * g.Hl + hl) * g.Nl + n;
+  // op 2: dst (b, hl, tok) <- [P] buffer (tok / Nl, b, tok % Nl, hl)
+  const long long b = i / (g.Hl * g.N), hl = (i / g.N) % g.Hl, tok = i % g.N;
+  const long long r = tok / g.Nl;
+  return p_row(g, r, b, tok - r * g.Nl, hl);
 }
 
 // Destination row of the i-th row of the dense destination enumeration.
 __device__ __forceinline__ long long dst_row(long long i, int op, const UlyGeom& g) {
-  if (op == 0 || op == 2) {  // the destination is the [P] buffer
-    const long long inner = g.B * g.Hl * g.Nl;
+  if (op == 0 || op == 3) {  // the destination is the [P] buffer
+    const long long inner = g.B * g.Nl * g.Hl;
     const long long r = i / inner;
     return g.base_rows + r * g.chunk_rows + (i - r * inner);
   }

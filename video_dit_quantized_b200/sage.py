@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "sage_linear_w8a16_workspace_bytes": (sz, [i32, i32]),
         "sage_linear_w8a16": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, vp]),
         "sage_ulysses_permute": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, ll, ll, vp]),
+        "sage_seqpar_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+        "sage_attn_fwd_seqpar": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]),
         "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
         "sage_dbg_mma_peak": (i32, [i32, i32, i32, vp, i32, vp, vp]),
         "sage_dbg_linear_bf16_forced_timeout": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
@@ -439,7 +441,7 @@ def linear_w8a16(x, wq, sw, bias=None, y=None, out_dtype=None, workspace=None, s
     return y
 
 
-ULYSSES_SEND_QKV, ULYSSES_RECV_QKV, ULYSSES_SEND_O, ULYSSES_RECV_O = 0, 1, 2, 3
+ULYSSES_SEND, ULYSSES_RECV_O, ULYSSES_GATHER, ULYSSES_SCATTER = 0, 1, 2, 3
 
 
 def host_chunk_heads(B: int, H: int, N: int, d: int) -> int:
@@ -457,7 +459,7 @@ def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, 
         raise ValueError(f"H={H} must be a multiple of P={P}")
     dense = B * (H // P) * Nl                     # rows of one [P] chunk
     p_side_rows = base_rows + (P - 1) * (chunk_rows or dense) + dense
-    chunked, flat = (dst, src) if op in (ULYSSES_SEND_QKV, ULYSSES_SEND_O) else (src, dst)
+    chunked, flat = (dst, src) if op in (ULYSSES_SEND, ULYSSES_SCATTER) else (src, dst)
     if flat.numel() < B * Nl * H * d:
         raise ValueError("the [B, ...] side holds fewer than B * Nl * H rows of d values")
     if chunked.numel() < p_side_rows * d:
@@ -465,6 +467,40 @@ def ulysses_permute(src, dst, B: int, Nl: int, H: int, d: int, P: int, op: int, 
     _check(LIB.sage_ulysses_permute(_dptr(src), _dptr(dst), B, Nl, H, d, P, op, int(chunk_rows), int(base_rows),
                                     _stream(stream)), "sage_ulysses_permute")
     return dst
+
+
+def seqpar_workspace_bytes(P: int, B: int, Nl: int, Hl: int, d: int, mode: int) -> int:
+    return int(LIB.sage_seqpar_workspace_bytes(P, B, Nl, Hl, d, mode))
+
+
+def alloc_seqpar_workspace(P: int, B: int, Nl: int, Hl: int, d: int, mode: int, device=None):
+    """Device workspace of sage_attn_fwd_seqpar (uint8, 256-byte aligned by the allocator)."""
+    import torch
+    n = seqpar_workspace_bytes(P, B, Nl, Hl, d, mode)
+    if n == 0:
+        raise SageError(EINVAL, "sage_seqpar_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+
+
+def attn_fwd_seqpar(q, k, v, mode: int, o=None, P: int = 1, workspace=None, stream=None):
+    """Attention on the sequence-parallel exchange layout: q, k, v, o bf16 [P, B, Nl, Hl, d] (chunk p:
+    tokens p*Nl .. p*Nl + Nl - 1, token-major).  Returns o."""
+    import torch
+    if q.dim() != 5 or q.shape[0] != P:
+        raise ValueError("q must be [P, B, Nl, Hl, d]")
+    shape = tuple(q.shape)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, shape)
+    _, B, Nl, Hl, d = shape
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", torch.bfloat16, shape)
+    if workspace is None:
+        workspace = alloc_seqpar_workspace(P, B, Nl, Hl, d, mode, q.device)
+    _check(LIB.sage_attn_fwd_seqpar(_dptr(q), _dptr(k), _dptr(v), _dptr(o), P, B, Nl, Hl, d, int(mode),
+                                    _dptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sage_attn_fwd_seqpar")
+    return o
 
 
 def status(workspace, stream=None) -> int:

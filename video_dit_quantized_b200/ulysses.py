@@ -7,15 +7,22 @@ kernels run unchanged on full sequences), and a second all-to-all returns
 the output to the sequence slices.  The all-to-all of q, k and v cost about
 2/3 of the attention time there, and the pages hide part of it by starting
 each exchange as soon as its tensor is computed, while the next projection
-still runs.  `UlyssesAttention.send` does exactly that: each of q, k, v is
-permuted into its send layout and its all-to-all is started at once
-(asynchronously, on the communicator's stream); `attend` waits for the three,
-runs the attention path on the local heads and brings O back.
+still runs.  `UlyssesAttention.send` does exactly that: each of q, k, v goes
+into its send layout and its all-to-all starts at once (asynchronously, on
+the communicator's stream); `attend` waits for the three, runs the attention
+path on the local heads and brings O back.
 
 Per rank: inputs [B, Nl, H, d] (this rank's Nl = N / P tokens, all heads),
-output [B, Nl, H, d].  The permutations are the C ABI's
-`sage_ulysses_permute`; the collectives are torch.distributed's
-`all_to_all_single` (NCCL on GPUs).
+output [B, Nl, H, d].  The exchange buffers are [P][B][Nl][Hl][d] (chunk r:
+this rank's tokens, heads r*Hl .. r*Hl + Hl - 1, token-major), so:
+  - at P = 1 the input already is the send layout and the receive buffer
+    already is the output: no data moves outside the collectives;
+  - at P > 1 the send copy and the O receive copy move contiguous runs of
+    Hl * d values (`sage_ulysses_permute`);
+  - the attention call `sage_attn_fwd_seqpar` reads q, k and v straight
+    from the receive buffers (the quantization prepass walks the chunks) and
+    writes O straight into the send buffer of the return exchange.
+The collectives are torch.distributed's `all_to_all_single` (NCCL on GPUs).
 """
 from __future__ import annotations
 
@@ -34,7 +41,8 @@ class UlyssesAttention:
     """One attention layer's Ulysses exchange for fixed shapes (buffers allocated once).
 
     permute(src, dst, B, Nl, H, d, P, op) and attention(q, k, v, mode, o, workspace) default to the
-    CUDA kernels; a2a(out, inp) -> handle defaults to an asynchronous all_to_all_single on `group`.
+    CUDA kernels (`attention` takes and gives the [P][B][Nl][Hl][d] exchange layout); a2a(out, inp)
+    -> handle defaults to an asynchronous all_to_all_single on `group`.
     """
 
     def __init__(self, B: int, Nl: int, H: int, d: int, world: int, mode: int = sage.MODE_INT8_FP8,
@@ -46,36 +54,45 @@ class UlyssesAttention:
         self.Hl, self.N = H // world, world * Nl
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         bf = torch.bfloat16
-        chunk = (world, B, self.Hl, Nl, d)
-        self.send_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"}
+        chunk = (world, B, Nl, self.Hl, d)
+        # at P = 1 the caller's tensor is sent as it is (same layout)
+        self.send_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"} if world > 1 else {}
         self.recv_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"}
-        self.local = {t: torch.empty((B, self.Hl, self.N, d), dtype=bf, device=dev) for t in "qkv"}
-        self.o_local = torch.empty((B, self.Hl, self.N, d), dtype=bf, device=dev)
         self.o_send = torch.empty(chunk, dtype=bf, device=dev)
         self.o_recv = torch.empty(chunk, dtype=bf, device=dev)
-        self.out = torch.empty((B, Nl, H, d), dtype=bf, device=dev)
+        self.out = torch.empty((B, Nl, H, d), dtype=bf, device=dev) if world > 1 else self.o_recv.view(B, Nl, H, d)
         self.workspace = None
         if attention is None and dev.type == "cuda":
-            self.workspace = sage.alloc_workspace(B, self.Hl, self.N, d, mode, dev)
+            self.workspace = sage.alloc_seqpar_workspace(world, B, Nl, self.Hl, d, mode, dev)
         self._permute = permute or (lambda src, dst, *g: sage.ulysses_permute(src, dst, *g))
-        self._attention = attention or (lambda q, k, v, m, o, ws: sage.attn_fwd(q, k, v, m, o=o, workspace=ws))
+        self._attention = attention or (
+            lambda q, k, v, m, o, ws: sage.attn_fwd_seqpar(q, k, v, m, o, world, workspace=ws))
         self._a2a = a2a or _default_a2a(group)
         self._pending = {}
+        self._keep = {}
 
     def _geom(self, op):
         return (self.B, self.Nl, self.H, self.d, self.P, op)
 
     def send(self, which: str, x):
-        """Start the exchange of q, k or v ([B, Nl, H, d] bf16): permute, then an async all-to-all."""
+        """Start the exchange of q, k or v ([B, Nl, H, d] bf16): send layout, then an async all-to-all.
+        At P = 1, x itself is sent: it must stay unchanged until attend_local()."""
         if which not in "qkv" or len(which) != 1:
             raise ValueError("which must be 'q', 'k' or 'v'")
         if tuple(x.shape) != (self.B, self.Nl, self.H, self.d):
             raise ValueError(f"{which} must be [B, Nl, H, d] = {(self.B, self.Nl, self.H, self.d)}")
-        self._permute(x.contiguous(), self.send_buf[which], *self._geom(sage.ULYSSES_SEND_QKV))
-        self._pending[which] = self._a2a(self.recv_buf[which], self.send_buf[which])
+        x = x.contiguous()
+        if self.P == 1:
+            src = x.view(1, self.B, self.Nl, self.H, self.d)
+            self._keep[which] = src
+        else:
+            src = self.send_buf[which]
+            self._permute(x, src, *self._geom(sage.ULYSSES_SEND))
+        self._pending[which] = self._a2a(self.recv_buf[which], src)
 
     def attend_local(self):
-        """Wait for q, k, v, run attention on the local heads and start O's way back."""
+        """Wait for q, k, v, run attention on the local heads (O lands in the send layout) and start
+        O's way back."""
         missing = [t for t in "qkv" if t not in self._pending]
         if missing:
             raise RuntimeError(f"send() was not called for {missing}")
@@ -83,9 +100,9 @@ class UlyssesAttention:
             h = self._pending.pop(t)
             if h is not None:
                 h.wait()
-            self._permute(self.recv_buf[t], self.local[t], *self._geom(sage.ULYSSES_RECV_QKV))
-        self._attention(self.local["q"], self.local["k"], self.local["v"], self.mode, self.o_local, self.workspace)
-        self._permute(self.o_local, self.o_send, *self._geom(sage.ULYSSES_SEND_O))
+        self._keep.clear()
+        self._attention(self.recv_buf["q"], self.recv_buf["k"], self.recv_buf["v"], self.mode, self.o_send,
+                        self.workspace)
         self._pending["o"] = self._a2a(self.o_recv, self.o_send)
 
     def finish(self):
@@ -93,7 +110,8 @@ class UlyssesAttention:
         h = self._pending.pop("o")
         if h is not None:
             h.wait()
-        self._permute(self.o_recv, self.out, *self._geom(sage.ULYSSES_RECV_O))
+        if self.P > 1:
+            self._permute(self.o_recv, self.out, *self._geom(sage.ULYSSES_RECV_O))
         return self.out
 
     def attend(self):
