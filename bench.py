@@ -62,17 +62,16 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "wan14b_720p"
-# Attention-kernel DRAM bytes (read + write) per full launch, from the ncu
-# captures summarised in profiles/attn_{i8f8,bf16}_wan14b_720p.md: a 4-head
-# capture of the same kernel, scaled by heads (each head's operands are read
-# from DRAM once).  Keyed by (workload, H, mode); absent keys report null.
+# Attention-kernel DRAM bytes (read + write) per full launch, from ncu captures
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the same kernels on 4 heads
+# of the same shape, scaled by heads (each head's operands are read from DRAM
+# once).  Keyed by (workload, H, mode); absent keys report null.
 NCU_TRAFFIC_BYTES = {
-    ("wan14b_720p", 40, "int8_fp8"): 1.653e9,
-    ("wan14b_720p", 40, "bf16"): 3.002e9,
+    ("wan14b_720p", 40, "int8_fp8"): 1.651e9,
+    ("wan14b_720p", 40, "bf16"): 3.006e9,
 }
-# Linear GEMM DRAM bytes per launch (ncu captures of the same kernels, summarised in
-# profiles/linear_{w8a8,bf16}_wan14b_720p.md), keyed by (workload, linear mode).
-# Absent keys report null.
+# Linear GEMM DRAM bytes per launch (ncu captures of the same kernels at the
+# same shape), keyed by (workload, linear mode).  Absent keys report null.
 NCU_TRAFFIC_BYTES_LINEAR = {
     ("wan14b_720p_proj", "w8a8"): 1.152e9,
     ("wan14b_720p_proj", "w8a16"): 3.477e9,
@@ -376,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
     # attention of another; every step moves all of Q, K, V in and all of O out.
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     chunk = sage.host_chunk_heads(w.B, w.H, w.N, w.d)
-    ws_e2e = sage.alloc_workspace(1, chunk, w.N, w.d, mode, dev)
+    ws_e2e = sage.alloc_host_workspace(w.B, w.H, w.N, w.d, mode, chunk, dev)
     staging = tuple(torch.empty_like(q) for _ in range(4))
     h2d = 3 * q.numel() * q.element_size()
     d2h = o.numel() * o.element_size()
@@ -441,7 +440,8 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * (2 if quant else 1),        # prepass (one persistent kernel) + attention
+        # prepass (statistics, finalize, quantize) + attention; BF16: attention only
+        "gpu_launches": args.steps * (4 if quant else 1),
         "mma_probe": {"kind": "i8" if quant else "bf16", "mac_per_clk_per_sm": probe["mac_per_clk_per_sm"],
                       "peak_at_median_sm_clock_tflops": (2 * probe["mac_per_clk_per_sm"] * probe["sms"] *
                                                          (clocks["sm_mhz"] or 0) * 1e6 / 1e12),
@@ -674,8 +674,8 @@ def run_ulysses(args, rank, world, local_rank):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
                    "parallelism": f"ulysses sp{world}", "tokens_per_rank": Nl, "heads_per_rank": w.H // world},
         # send copies of q, k, v and the O receive copy (none at P = 1: the layouts coincide), then the
-        # fused prepass + attention (BF16: three gathers + attention)
-        "gpu_launches": args.steps * ((4 if world > 1 else 0) + (2 if mode != sage.MODE_BF16 else 4)),
+        # prepass (three kernels) + attention (BF16: three gathers + attention)
+        "gpu_launches": args.steps * ((4 if world > 1 else 0) + 4),
         "clocks": clk.summary(),
     }), flush=True)
 
@@ -749,7 +749,7 @@ def run_stack(args, rank, world, local_rank):
     # its O back to pinned host memory
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     chunk = sage.host_chunk_heads(base.B, base.H, base.N, base.d)
-    ws_e2e = sage.alloc_workspace(1, chunk, base.N, base.d, sage.MODE_INT8_FP8, dev)
+    ws_e2e = sage.alloc_host_workspace(base.B, base.H, base.N, base.d, sage.MODE_INT8_FP8, chunk, dev)
     staging = tuple(torch.empty_like(o) for _ in range(4))
 
     def e2e_stack():
@@ -797,7 +797,7 @@ def run_stack(args, rank, world, local_rank):
                            "speedup_of_selective": ms_bf16 / ms, "clocks": clocks_bf16},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * sum(2 if m != sage.MODE_BF16 else 1 for m in modes),
+        "gpu_launches": args.steps * sum(4 if m != sage.MODE_BF16 else 1 for m in modes),
         "clocks": clocks,
     }), flush=True)
 

@@ -185,20 +185,34 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
  * q_host, k_host, v_host, o_host: HOST bf16 [B,H,N,d]; pinned (page-locked)
  *   memory is needed for the copies to overlap.
  * q_dev, k_dev, v_dev, o_dev: device staging buffers bf16 [B,H,N,d] (caller-owned).
- * workspace: at least sage_workspace_bytes(1, chunk_heads, N, d, mode) bytes,
- *   reused by every chunk.
+ * workspace: at least sage_host_workspace_bytes(B, H, N, d, mode, chunk_heads)
+ *   bytes, zero-filled before the first call: its two halves (each rounded
+ *   down to 256 bytes; one when B*H == 1) are the workspaces of alternate
+ *   chunks, each with its status word first, at the same offsets whatever the
+ *   mode, so one buffer serves calls of every mode.
  * The first and the last chunk take half as many heads (at least one): they
- * are the copies nothing overlaps.
+ * are the copies nothing overlaps.  Alternate chunks run on `stream` and on a
+ * second compute stream, so one chunk's prepass and attention start while
+ * the previous chunk's last wave drains.
  * Runs after earlier work on `stream` and returns when the output is in
- * o_host (it synchronises).  Its two copy streams and three events are made
- * on the first call on a device (and again in a new CUDA context) and kept
- * until the process exits; calls on one device from several host threads run
- * one after the other.  Allocates no device memory.  Returns the status of
- * the call including device-side status (SAGE_ETIMEOUT).
+ * o_host (it synchronises).  Its three streams (copy in, copy out, second
+ * compute stream) and three events are made on the first call on a device
+ * (and again in a new CUDA context) and kept until the process exits; calls
+ * on one device from several host threads run one after the other.
+ * Allocates no device memory.  Returns the status of the call including
+ * device-side status (SAGE_ETIMEOUT).
  */
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H,
                        int N, int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
                        void* workspace, size_t workspace_bytes, int chunk_heads, void* stream);
+
+/*
+ * Workspace bytes of sage_attn_fwd_host for this shape, mode and chunk
+ * (chunk_heads 0: sage_host_chunk_heads()): two 256-byte aligned copies of
+ * sage_workspace_bytes(1, chunk_heads, N, d, mode) (one when B*H == 1).
+ * 0 on a bad shape or mode.
+ */
+size_t sage_host_workspace_bytes(int B, int H, int N, int d, int mode, int chunk_heads);
 
 /*
  * The default chunk of sage_attn_fwd_host: the fewest heads whose attention

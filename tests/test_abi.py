@@ -14,7 +14,7 @@ EXPECTED = {
     "sage_select_full_precision_layers", "sage_quantize_qk_ex", "sage_attn_quantized_ex",
     "sage_quantize_blocks_2d", "sage_linear_w8a8", "sage_dbg_linear_forced_timeout",
     "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
-    "sage_ulysses_permute", "sage_host_chunk_heads", "sage_dbg_mma_peak", "sage_dbg_linear_bf16_forced_timeout",
+    "sage_ulysses_permute", "sage_host_chunk_heads", "sage_host_workspace_bytes", "sage_dbg_mma_peak", "sage_dbg_linear_bf16_forced_timeout",
     "sage_attn_rel_l2", "sage_seqpar_workspace_bytes", "sage_attn_fwd_seqpar",
 }
 

@@ -35,3 +35,28 @@ def test_host_pipeline_rejects_small_workspace(cuda_dev):
     with pytest.raises(sage.SageError) as e:
         sage.attn_fwd_host(qh, kh, vh, oh, sage.MODE_INT8_FP8, workspace=ws, chunk_heads=1)
     assert e.value.code == sage.EWORKSPACE
+    # one chunk's workspace is not enough: two chunks are in flight
+    one = sage.workspace_bytes(1, 1, w.N, w.d, sage.MODE_INT8_FP8)
+    assert sage.host_workspace_bytes(w.B, w.H, w.N, w.d, sage.MODE_INT8_FP8, 1) == 2 * ((one + 255) // 256 * 256)
+    ws = torch.zeros(one, dtype=torch.uint8, device=cuda_dev)
+    with pytest.raises(sage.SageError) as e:
+        sage.attn_fwd_host(qh, kh, vh, oh, sage.MODE_INT8_FP8, workspace=ws, chunk_heads=1)
+    assert e.value.code == sage.EWORKSPACE
+
+
+def test_host_pipeline_one_workspace_for_every_mode(cuda_dev):
+    """A layer stack alternates modes on one host workspace (sized for INT8/FP8): every call must
+    find its chunks' status words where the previous call of another mode left them clean."""
+    import torch
+    from video_dit_quantized_b200 import sage
+    w = synth.Workload("stackmix", 1, 6, 1100, 128, seed=63)
+    qh, kh, vh = synth.qkv_torch(w, pin=True)
+    qd, kd, vd = (t.to(cuda_dev) for t in (qh, kh, vh))
+    ws = sage.alloc_host_workspace(w.B, w.H, w.N, w.d, sage.MODE_INT8_FP8, 2, cuda_dev)
+    staging = tuple(torch.empty(qh.shape, dtype=torch.bfloat16, device=cuda_dev) for _ in range(4))
+    for mode in (sage.MODE_INT8_FP8, sage.MODE_BF16, sage.MODE_INT8_FP8, sage.MODE_INT8_FP8_QTOKEN, sage.MODE_BF16):
+        ref = sage.attn_fwd(qd, kd, vd, mode)
+        oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+        sage.attn_fwd_host(qh, kh, vh, oh, mode, staging=staging, workspace=ws, chunk_heads=2)
+        torch.cuda.synchronize()
+        assert torch.equal(oh.view(torch.int16), ref.cpu().view(torch.int16)), mode

@@ -109,6 +109,9 @@ def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
 
     def exchange():
         # rank r receives chunk r of every rank's send buffer, in rank order
+        # (one rank sends nothing: its exchange is the identity)
+        if not sent:
+            return
         outs = {}
         for (r, _), (out, inp) in sent.items():
             outs.setdefault(r, []).append((out, inp))
@@ -133,7 +136,9 @@ def test_emulated_ranks_equal_one_call(mode_name, P, cuda_dev):
 
 
 def test_single_rank_nccl_exchange(cuda_dev):
-    """The default communicator path: a one-rank NCCL group, all_to_all_single as the exchange."""
+    """A one-rank NCCL group: the layer runs with no collective (the exchange of one rank is the
+    identity) and equals one attention call; the default exchange itself, an asynchronous
+    all_to_all_single on the group, moves a buffer in the layer's send layout unchanged."""
     import os
     import socket
 
@@ -157,6 +162,12 @@ def test_single_rank_nccl_exchange(cuda_dev):
         out = ua(*(t.permute(0, 2, 1, 3).contiguous() for t in (q, k, v)))
         torch.cuda.synchronize()
         assert torch.equal(out.permute(0, 2, 1, 3).contiguous().view(torch.int16), ref.view(torch.int16))
+        from video_dit_quantized_b200.ulysses import _default_a2a
+        src = q.permute(0, 2, 1, 3).contiguous().view(1, w.B, w.N, w.H, w.d)
+        dst = torch.empty_like(src)
+        _default_a2a(None)(dst, src).wait()
+        torch.cuda.synchronize()
+        assert torch.equal(dst.view(torch.int16), src.view(torch.int16))
     finally:
         if group_made:
             dist.destroy_process_group()

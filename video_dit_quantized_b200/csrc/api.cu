@@ -62,7 +62,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct HostPipe {
   std::mutex mu;
   unsigned long long ctx = 0;
-  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_alt = nullptr;
   cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_done = nullptr;
 };
 constexpr int kMaxHostDevices = 64;
@@ -74,20 +74,22 @@ bool pipe_ready(HostPipe& p) {
   const unsigned long long ctx = current_context_id();
   if (p.s_in && ctx != 0 && ctx == p.ctx) return true;
   // handles of an earlier context are gone with it
-  p.s_in = p.s_out = nullptr;
+  p.s_in = p.s_out = p.s_alt = nullptr;
   p.ev_start = p.ev_in = p.ev_done = nullptr;
   bool ok = cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.s_alt, cudaStreamNonBlocking) == cudaSuccess &&
             cudaEventCreateWithFlags(&p.ev_start, cudaEventDisableTiming) == cudaSuccess &&
             cudaEventCreateWithFlags(&p.ev_in, cudaEventDisableTiming) == cudaSuccess &&
             cudaEventCreateWithFlags(&p.ev_done, cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
     if (p.s_in) cudaStreamDestroy(p.s_in);
     if (p.s_out) cudaStreamDestroy(p.s_out);
+    if (p.s_alt) cudaStreamDestroy(p.s_alt);
     if (p.ev_start) cudaEventDestroy(p.ev_start);
     if (p.ev_in) cudaEventDestroy(p.ev_in);
     if (p.ev_done) cudaEventDestroy(p.ev_done);
-    p.s_in = p.s_out = nullptr;
+    p.s_in = p.s_out = p.s_alt = nullptr;
     p.ev_start = p.ev_in = p.ev_done = nullptr;
     return false;
   }
@@ -341,6 +343,16 @@ int sage_host_chunk_heads(int B, int H, int N, int d) {
   return (int)chunk;
 }
 
+size_t sage_host_workspace_bytes(int B, int H, int N, int d, int mode, int chunk_heads) {
+  if (check_shape(B, H, N, d) != SAGE_OK) return 0;
+  if (mode != SAGE_MODE_BF16 && mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_INT8_FP8_QTOKEN) return 0;
+  const int BH = B * H;
+  if (chunk_heads <= 0) chunk_heads = sage_host_chunk_heads(B, H, N, d);
+  if (chunk_heads > BH) chunk_heads = BH;
+  const size_t one = align_up(sage_workspace_bytes(1, chunk_heads, N, d, mode), 256);
+  return BH > 1 ? 2 * one : one;      // two chunks in flight, one workspace each
+}
+
 int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, int B, int H, int N,
                        int d, int mode, void* q_dev, void* k_dev, void* v_dev, void* o_dev, void* workspace,
                        size_t workspace_bytes, int chunk_heads, void* stream) {
@@ -353,8 +365,12 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   const int BH = B * H;
   if (chunk_heads <= 0) chunk_heads = sage_host_chunk_heads(B, H, N, d);
   if (chunk_heads > BH) chunk_heads = BH;
-  const int n_chunks = (BH + chunk_heads - 1) / chunk_heads;
-  if (workspace_bytes < sage_workspace_bytes(1, chunk_heads, N, d, mode)) return SAGE_EWORKSPACE;
+  if (workspace_bytes < sage_host_workspace_bytes(B, H, N, d, mode, chunk_heads)) return SAGE_EWORKSPACE;
+  // The two chunk workspaces split the buffer in halves whatever the mode, so
+  // their status words sit at the same places for every call on one buffer
+  // (a layer stack alternates modes on the same workspace).
+  const int n_ws = BH > 1 ? 2 : 1;
+  const size_t ws_one = n_ws == 2 ? (workspace_bytes / 2) & ~size_t(255) : workspace_bytes;
   if ((rc = check_device()) != SAGE_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int dev = 0;
@@ -364,10 +380,16 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   if (!pipe_ready(pipe)) return SAGE_ELAUNCH;
   cudaStream_t s_in = pipe.s_in, s_out = pipe.s_out;
   cudaEvent_t ev_start = pipe.ev_start, ev_in = pipe.ev_in, ev_done = pipe.ev_done;
-  // inputs of chunk i land (s_in) -> its attention runs (stream) -> its output leaves (s_out);
-  // copies may not start before earlier work on the caller's stream
+  // Chunks alternate between the caller's stream and a second compute stream,
+  // each with its own half of the workspace, so that chunk i+1's prepass and
+  // the start of its attention fill the SMs that chunk i's last wave leaves
+  // idle.  Inputs of chunk i land (s_in) -> its prepass and attention run
+  // (compute stream i % 2) -> its output leaves (s_out).  Nothing starts
+  // before earlier work on the caller's stream.
+  cudaStream_t s_comp[2] = {st, pipe.s_alt};
   cudaEventRecord(ev_start, st);
   cudaStreamWaitEvent(s_in, ev_start, 0);
+  cudaStreamWaitEvent(pipe.s_alt, ev_start, 0);
   const size_t head_bytes = (size_t)N * d * 2;
   const char* qh = static_cast<const char*>(q_host);
   const char* kh = static_cast<const char*>(k_host);
@@ -377,36 +399,47 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   char* kd = static_cast<char*>(k_dev);
   char* vd = static_cast<char*>(v_dev);
   char* od = static_cast<char*>(o_dev);
+  char* ws = static_cast<char*>(workspace);
   // The first and the last chunk take half as many heads: the first upload and
   // the last download are the parts of the pipeline nothing overlaps.
   const int half = std::max(1, chunk_heads / 2);
   const int first = std::min(half, BH);
   const int last = std::min(half, BH - first);
   rc = SAGE_OK;
-  for (int h0 = 0; h0 < BH && rc == SAGE_OK;) {
+  int i = 0;
+  for (int h0 = 0; h0 < BH && rc == SAGE_OK; ++i) {
     int hc = h0 == 0 ? first : std::min(chunk_heads, BH - last - h0);
     if (hc <= 0) hc = BH - h0;                       // the last chunk
     const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hc * head_bytes;
+    cudaStream_t sc = s_comp[i % n_ws];
+    char* wsi = ws + (size_t)(i % n_ws) * ws_one;
     if (cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
         cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
         cudaMemcpyAsync(vd + off, vh + off, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(st, ev_in, 0) != cudaSuccess) {
+        cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(sc, ev_in, 0) != cudaSuccess) {
       rc = SAGE_ELAUNCH;
       break;
     }
-    rc = sage_attn_fwd(qd + off, kd + off, vd + off, od + off, 1, hc, N, d, mode, workspace, workspace_bytes, stream);
+    rc = sage_attn_fwd(qd + off, kd + off, vd + off, od + off, 1, hc, N, d, mode, wsi, ws_one, sc);
     if (rc != SAGE_OK) break;
-    if (cudaEventRecord(ev_done, st) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
+    if (cudaEventRecord(ev_done, sc) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done, 0) != cudaSuccess ||
         cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
       rc = SAGE_ELAUNCH;
     h0 += hc;
   }
-  // the caller's stream resumes after the last output copy
+  // every chunk's compute precedes its output copy on s_out, so the caller's
+  // stream resumes after the last output copy
   cudaEventRecord(ev_done, s_out);
   cudaStreamWaitEvent(st, ev_done, 0);
-  if (cudaStreamSynchronize(s_out) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) rc = SAGE_ELAUNCH;
+  if (cudaStreamSynchronize(s_out) != cudaSuccess || cudaStreamSynchronize(pipe.s_alt) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    rc = SAGE_ELAUNCH;
   if (rc != SAGE_OK) return rc;
-  return sage_status(workspace, stream);
+  for (int w = 0; w < n_ws; ++w) {
+    const int r = sage_status(ws + (size_t)w * ws_one, stream);
+    if (r != SAGE_OK) rc = r;
+  }
+  return rc;
 }
 
 int attn_layer_schedule(int num_layers, const int* full_precision_layers, int n_fp, int8_t* modes_out) {

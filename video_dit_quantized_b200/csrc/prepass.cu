@@ -61,7 +61,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
-// grid (nK, BH).  TOKQ: Q gets one scale per token (q_scale [BH, Npad]) instead
+// grid (nK, BH), or (nK * BH) with the head fastest when CHUNKED.  TOKQ: Q gets one scale per token (q_scale [BH, Npad]) instead
 // of one per 128-token block (q_scale [BH, nK]).
 template <int D, bool TOKQ, bool CHUNKED>
 __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __restrict__ q,
@@ -77,7 +77,12 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
   __shared__ int vamax_s[D];                       // non-negative floats as int bits
   __shared__ float red[kThreads / 32];
 
-  const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
+  // chunked layout: a 1-D grid, head fastest, so that the CTAs resident at one
+  // time read the same token tile of every local head, one contiguous range
+  const int BHc = CHUNKED ? in_map.B * in_map.Hl : 1;
+  const int kb = CHUNKED ? (int)(blockIdx.x / BHc) : (int)blockIdx.x;
+  const int bh = CHUNKED ? (int)(blockIdx.x % BHc) : (int)blockIdx.y;
+  const int nK = CHUNKED ? (int)(gridDim.x / BHc) : (int)gridDim.x;
   const int n0 = kb * kTile;
   const int nr = min(kTile, N - n0);
   const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
@@ -170,24 +175,67 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
   }
 }
 
-// grid (BH), block D
+// grid (BH, D / 32), block 64.  Warp 0 adds the K partial sums of 32
+// channels in ascending block order (the fp64 order of the K mean), warp 1
+// takes the V absmax of the same channels.  Each lane walks its channel's
+// column of partials (a warp reads 32 consecutive channels of one block per
+// load, 256 or 128 contiguous bytes) with the next kFinBatch blocks' loads in
+// flight while it adds the current ones, so the chain of additions, not the
+// load latency, sets the time.
+constexpr int kFinBatch = 32;
 template <int D>
-__global__ void prepass_finalize_kernel(int N, int nK, PrepassScratch scr, float* __restrict__ k_mean,
-                                        float* __restrict__ v_scale) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  double total = 0.0;
-  float a = 0.f;
-  for (int t = 0; t < nK; ++t) {
-    const size_t idx = ((size_t)bh * nK + t) * D + c;
-    total = __dadd_rn(total, scr.k_psum[idx]);
-    a = fmaxf(a, scr.v_pamax[idx]);
+__global__ void __launch_bounds__(64) prepass_finalize_kernel(int N, int nK, PrepassScratch scr,
+                                                              float* __restrict__ k_mean,
+                                                              float* __restrict__ v_scale) {
+  const int bh = blockIdx.x;
+  const int c = blockIdx.y * 32 + (threadIdx.x & 31);
+  const size_t col = (size_t)bh * nK * D + c;       // partial (bh, block 0, c); block t is t * D further
+  if (threadIdx.x < 32) {
+    const double* gs = scr.k_psum + col;
+    double total = 0.0;
+    double A[kFinBatch], B[kFinBatch];
+    auto load = [&](double(&r)[kFinBatch], int t0) {
+#pragma unroll
+      for (int i = 0; i < kFinBatch; ++i) r[i] = t0 + i < nK ? gs[(size_t)(t0 + i) * D] : 0.0;
+    };
+    auto add = [&](const double(&r)[kFinBatch], int t0) {
+#pragma unroll
+      for (int i = 0; i < kFinBatch; ++i)
+        if (t0 + i < nK) total = __dadd_rn(total, r[i]);
+    };
+    load(A, 0);
+    for (int t0 = 0; t0 < nK; t0 += 2 * kFinBatch) {
+      load(B, t0 + kFinBatch);
+      add(A, t0);
+      load(A, t0 + 2 * kFinBatch);
+      add(B, t0 + kFinBatch);
+    }
+    k_mean[(size_t)bh * D + c] = __double2float_rn(__ddiv_rn(total, (double)N));
+  } else {
+    const float* ga = scr.v_pamax + col;
+    float a = 0.f;
+    float A[kFinBatch], B[kFinBatch];
+    auto load = [&](float(&r)[kFinBatch], int t0) {
+#pragma unroll
+      for (int i = 0; i < kFinBatch; ++i) r[i] = t0 + i < nK ? ga[(size_t)(t0 + i) * D] : 0.f;
+    };
+    auto take = [&](const float(&r)[kFinBatch]) {
+#pragma unroll
+      for (int i = 0; i < kFinBatch; ++i) a = fmaxf(a, r[i]);   // absmax partials are >= 0; padding adds 0
+    };
+    load(A, 0);
+    for (int t0 = 0; t0 < nK; t0 += 2 * kFinBatch) {
+      load(B, t0 + kFinBatch);
+      take(A);
+      load(A, t0 + 2 * kFinBatch);
+      take(B);
+    }
+    v_scale[(size_t)bh * D + c] = a > 0.f ? __fdiv_rn(a, 448.0f) : 0.f;
+    scr.v_amax[(size_t)bh * D + c] = a;
   }
-  k_mean[(size_t)bh * D + c] = __double2float_rn(__ddiv_rn(total, (double)N));
-  v_scale[(size_t)bh * D + c] = a > 0.f ? __fdiv_rn(a, 448.0f) : 0.f;
-  scr.v_amax[(size_t)bh * D + c] = a;
 }
 
-// grid (nK, BH)
+// grid (nK, BH), or (nK * BH) with the head fastest when CHUNKED
 template <int D, bool CHUNKED>
 __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4* __restrict__ k,
                                                                     const uint4* __restrict__ v, int N, int Npad,
@@ -203,7 +251,12 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   __shared__ __align__(16) uint4 vs[kTile * V8];
   __shared__ float red[kThreads / 32];
 
-  const int kb = blockIdx.x, bh = blockIdx.y, nK = gridDim.x;
+  // chunked layout: a 1-D grid, head fastest, so that the CTAs resident at one
+  // time read the same token tile of every local head, one contiguous range
+  const int BHc = CHUNKED ? in_map.B * in_map.Hl : 1;
+  const int kb = CHUNKED ? (int)(blockIdx.x / BHc) : (int)blockIdx.x;
+  const int bh = CHUNKED ? (int)(blockIdx.x % BHc) : (int)blockIdx.y;
+  const int nK = CHUNKED ? (int)(gridDim.x / BHc) : (int)gridDim.x;
   const int n0 = kb * kTile;
   const int nr = min(kTile, N - n0);
   const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
@@ -279,11 +332,12 @@ cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH
                              float* v_scale, const PrepassScratch& scr, bool q_per_token, cudaStream_t stream,
                              RowMap in_map) {
   const int nK = num_tiles(N), Npad = nK * kTile;
-  dim3 grid(nK, BH);
+  const bool chunked = in_map.P != 0;
+  if (chunked && in_map.B * in_map.Hl != BH) return cudaErrorInvalidValue;
+  const dim3 grid = chunked ? dim3((unsigned)nK * BH) : dim3(nK, BH);
   const uint4* q4 = static_cast<const uint4*>(q);
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
-  const bool chunked = in_map.P != 0;
   if (q_per_token && chunked)
     prepass_stats_kernel<D, true, true><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
   else if (q_per_token)
@@ -292,7 +346,7 @@ cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH
     prepass_stats_kernel<D, false, true><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
   else
     prepass_stats_kernel<D, false, false><<<grid, kThreads, 0, stream>>>(q4, k4, v4, N, Npad, q_i8, q_scale, scr, in_map);
-  prepass_finalize_kernel<D><<<BH, D, 0, stream>>>(N, nK, scr, k_mean, v_scale);
+  prepass_finalize_kernel<D><<<dim3(BH, D / 32), 64, 0, stream>>>(N, nK, scr, k_mean, v_scale);
   if (chunked)
     prepass_quant_kv_kernel<D, true><<<grid, kThreads, 0, stream>>>(k4, v4, N, Npad, k_mean, k_i8, k_scale, v_f8t, scr,
                                                                     in_map);

@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "sage_seqpar_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "sage_attn_fwd_seqpar": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]),
         "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
+        "sage_host_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
         "sage_dbg_mma_peak": (i32, [i32, i32, i32, vp, i32, vp, vp]),
         "sage_dbg_linear_bf16_forced_timeout": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
     }
@@ -149,6 +150,19 @@ def workspace_bytes(B: int, H: int, N: int, d: int, mode: int) -> int:
 
 def prepass_scratch_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(LIB.sage_prepass_scratch_bytes(B, H, N, d))
+
+
+def host_workspace_bytes(B: int, H: int, N: int, d: int, mode: int, chunk_heads: int = 0) -> int:
+    return int(LIB.sage_host_workspace_bytes(B, H, N, d, int(mode), int(chunk_heads)))
+
+
+def alloc_host_workspace(B: int, H: int, N: int, d: int, mode: int, chunk_heads: int = 0, device=None):
+    """Zero-filled workspace of attn_fwd_host (two chunk workspaces)."""
+    import torch
+    n = host_workspace_bytes(B, H, N, d, mode, chunk_heads)
+    if n == 0:
+        raise SageError(EINVAL, "sage_host_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def alloc_workspace(B: int, H: int, N: int, d: int, mode: int, device=None):
@@ -238,7 +252,8 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, c
     """sage_attn_fwd_host: host bf16 [B,H,N,d] tensors (pinned for overlap) in, o_h filled on return.
 
     staging: optional tuple of four device bf16 tensors shaped like q_h; workspace: optional
-    device buffer of sage_workspace_bytes(1, chunk, N, d, mode) bytes.
+    zero-filled device buffer of sage_host_workspace_bytes(B, H, N, d, mode, chunk) bytes
+    (alloc_host_workspace).
     """
     import torch
     B, H, N, d = _bhnd(q_h, "q_h")
@@ -248,7 +263,7 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, mode: int, staging=None, workspace=None, c
     if staging is None:
         staging = tuple(torch.empty(q_h.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
     if workspace is None:
-        workspace = alloc_workspace(1, chunk, N, d, mode)
+        workspace = alloc_host_workspace(B, H, N, d, mode, chunk)
     qd, kd, vd, od = staging
     _check(LIB.sage_attn_fwd_host(_ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(o_h), B, H, N, d, int(mode), _dptr(qd),
                                   _dptr(kd), _dptr(vd), _dptr(od), _dptr(workspace),

@@ -15,8 +15,9 @@ path on the local heads and brings O back.
 Per rank: inputs [B, Nl, H, d] (this rank's Nl = N / P tokens, all heads),
 output [B, Nl, H, d].  The exchange buffers are [P][B][Nl][Hl][d] (chunk r:
 this rank's tokens, heads r*Hl .. r*Hl + Hl - 1, token-major), so:
-  - at P = 1 the input already is the send layout and the receive buffer
-    already is the output: no data moves outside the collectives;
+  - at P = 1 the input already is the send layout and the exchange of one
+    rank is the identity: attention reads the inputs and writes the output
+    in place, and no collective runs;
   - at P > 1 the send copy and the O receive copy move contiguous runs of
     Hl * d values (`sage_ulysses_permute`);
   - the attention call `sage_attn_fwd_seqpar` reads q, k and v straight
@@ -56,11 +57,12 @@ class UlyssesAttention:
         bf = torch.bfloat16
         chunk = (world, B, Nl, self.Hl, d)
         # at P = 1 the caller's tensor is sent as it is (same layout)
-        self.send_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"} if world > 1 else {}
-        self.recv_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"}
+        multi = world > 1
+        self.send_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"} if multi else {}
+        self.recv_buf = {t: torch.empty(chunk, dtype=bf, device=dev) for t in "qkv"} if multi else {}
         self.o_send = torch.empty(chunk, dtype=bf, device=dev)
-        self.o_recv = torch.empty(chunk, dtype=bf, device=dev)
-        self.out = torch.empty((B, Nl, H, d), dtype=bf, device=dev) if world > 1 else self.o_recv.view(B, Nl, H, d)
+        self.o_recv = torch.empty(chunk, dtype=bf, device=dev) if multi else self.o_send
+        self.out = torch.empty((B, Nl, H, d), dtype=bf, device=dev) if multi else self.o_send.view(B, Nl, H, d)
         self.workspace = None
         if attention is None and dev.type == "cuda":
             self.workspace = sage.alloc_seqpar_workspace(world, B, Nl, self.Hl, d, mode, dev)
@@ -83,11 +85,12 @@ class UlyssesAttention:
             raise ValueError(f"{which} must be [B, Nl, H, d] = {(self.B, self.Nl, self.H, self.d)}")
         x = x.contiguous()
         if self.P == 1:
-            src = x.view(1, self.B, self.Nl, self.H, self.d)
-            self._keep[which] = src
-        else:
-            src = self.send_buf[which]
-            self._permute(x, src, *self._geom(sage.ULYSSES_SEND))
+            # the exchange of one rank is the identity: attention reads x itself
+            self._keep[which] = x.view(1, self.B, self.Nl, self.H, self.d)
+            self._pending[which] = None
+            return
+        src = self.send_buf[which]
+        self._permute(x, src, *self._geom(sage.ULYSSES_SEND))
         self._pending[which] = self._a2a(self.recv_buf[which], src)
 
     def attend_local(self):
@@ -100,10 +103,10 @@ class UlyssesAttention:
             h = self._pending.pop(t)
             if h is not None:
                 h.wait()
-        self._keep.clear()
-        self._attention(self.recv_buf["q"], self.recv_buf["k"], self.recv_buf["v"], self.mode, self.o_send,
-                        self.workspace)
-        self._pending["o"] = self._a2a(self.o_recv, self.o_send)
+        src = self._keep if self.P == 1 else self.recv_buf
+        self._attention(src["q"], src["k"], src["v"], self.mode, self.o_send, self.workspace)
+        self._keep = {}
+        self._pending["o"] = self._a2a(self.o_recv, self.o_send) if self.P > 1 else None
 
     def finish(self):
         """Wait for O and return it for this rank's tokens, [B, Nl, H, d]."""
