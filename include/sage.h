@@ -54,6 +54,7 @@ extern "C" {
 #define SAGE_ELAUNCH (-3)       /* a CUDA launch or runtime call failed               */
 #define SAGE_EWORKSPACE (-4)    /* workspace smaller than sage_workspace_bytes()      */
 #define SAGE_ETIMEOUT (-5)      /* a bounded device-side wait ran out (see sage_status) */
+#define SAGE_EBOUNDS (-6)       /* a device-side bounds check failed (debug build only) */
 
 /* tile sizes of the quantization blocks and of the attention tiles */
 #define SAGE_BLK_Q 128
@@ -407,6 +408,30 @@ const char* sage_strerror(int code);
  * built for, SAGE_EUNSUPPORTED otherwise, SAGE_ELAUNCH if no device is usable.
  */
 int sage_device_check(void);
+
+/*
+ * Debug build.  The same sources compiled with -DSAGE_DEBUG give
+ * libsage_debug.so: every global access of the prepass, of the attention
+ * kernels' scale loads and output stores, and of the Ulysses permutations
+ * whose index is computed is checked against the extent of its buffer
+ * first.  A failed check skips that access and records the site and the
+ * index of the first failure; nothing traps.  The device entry points of the
+ * quantization path, attention and the permutations then synchronise their
+ * stream and return SAGE_EBOUNDS if a check failed (so a debug build cannot
+ * be captured into a CUDA graph).  A release build has no checks.
+ *
+ * sage_debug_build: 1 in a debug build, 0 otherwise.
+ * sage_debug_last_failure: the site (see csrc/internal.h, DebugSite) and the
+ *   index of the first failed check of the last call that returned
+ *   SAGE_EBOUNDS; SAGE_EUNSUPPORTED in a release build.
+ * sage_dbg_bounds_selftest: runs a one-thread kernel whose single check
+ *   fails on purpose (the index equals the extent; no memory is touched) and
+ *   returns what a call with a failed check returns: SAGE_EBOUNDS in a debug
+ *   build (site 99, index 1); SAGE_EUNSUPPORTED in a release build.
+ */
+int sage_debug_build(void);
+int sage_debug_last_failure(int* site, long long* index);
+int sage_dbg_bounds_selftest(void* stream);
 
 /*
  * Diagnostic: copies int32 QK^T tiles computed by the same TMA + tcgen05

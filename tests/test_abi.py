@@ -16,6 +16,7 @@ EXPECTED = {
     "sage_dequant_blocks_2d", "sage_linear_bf16", "sage_linear_w8a16_workspace_bytes", "sage_linear_w8a16",
     "sage_ulysses_permute", "sage_host_chunk_heads", "sage_host_workspace_bytes", "sage_dbg_mma_peak", "sage_dbg_linear_bf16_forced_timeout",
     "sage_attn_rel_l2", "sage_seqpar_workspace_bytes", "sage_attn_fwd_seqpar",
+    "sage_debug_build", "sage_debug_last_failure", "sage_dbg_bounds_selftest",
 }
 
 
@@ -27,6 +28,22 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(sage._build.LIB_PATH)
     for name in sage.header_functions():
         assert hasattr(lib, name), name
+
+
+def test_debug_build_exports_the_same_symbols_and_says_it_is_one():
+    dbg = sage.debug_library()
+    for name in sage.header_functions():
+        assert hasattr(dbg, name), name
+    assert sage.LIB.sage_debug_build() == 0 and dbg.sage_debug_build() == 1
+    site, index = ctypes.c_int(-1), ctypes.c_longlong(-1)
+    # a release build keeps no failure record; a debug build has none yet
+    assert sage.LIB.sage_debug_last_failure(ctypes.byref(site), ctypes.byref(index)) == sage.EUNSUPPORTED
+    assert dbg.sage_debug_last_failure(ctypes.byref(site), ctypes.byref(index)) == sage.OK
+    assert (site.value, index.value) == (0, 0)
+    assert dbg.sage_debug_last_failure(None, None) == sage.EINVAL
+    # the release self-test has no check to fail; neither touches a device before that answer
+    assert sage.LIB.sage_dbg_bounds_selftest(None) == sage.EUNSUPPORTED
+    assert sage.strerror(sage.EBOUNDS) == "a device-side bounds check failed (debug build)"
 
 
 def test_workspace_sizes():

@@ -45,14 +45,15 @@ def test_host_pipeline_rejects_small_workspace(cuda_dev):
 
 
 def test_host_pipeline_one_workspace_for_every_mode(cuda_dev):
-    """A layer stack alternates modes on one host workspace (sized for INT8/FP8): every call must
-    find its chunks' status words where the previous call of another mode left them clean."""
+    """A layer stack alternates modes on one host workspace (sized for the largest mode, per-token
+    INT8/FP8): every call must find its chunks' status words where the previous call of another mode
+    left them clean."""
     import torch
     from video_dit_quantized_b200 import sage
     w = synth.Workload("stackmix", 1, 6, 1100, 128, seed=63)
     qh, kh, vh = synth.qkv_torch(w, pin=True)
     qd, kd, vd = (t.to(cuda_dev) for t in (qh, kh, vh))
-    ws = sage.alloc_host_workspace(w.B, w.H, w.N, w.d, sage.MODE_INT8_FP8, 2, cuda_dev)
+    ws = sage.alloc_host_workspace(w.B, w.H, w.N, w.d, sage.MODE_INT8_FP8_QTOKEN, 2, cuda_dev)
     staging = tuple(torch.empty(qh.shape, dtype=torch.bfloat16, device=cuda_dev) for _ in range(4))
     for mode in (sage.MODE_INT8_FP8, sage.MODE_BF16, sage.MODE_INT8_FP8, sage.MODE_INT8_FP8_QTOKEN, sage.MODE_BF16):
         ref = sage.attn_fwd(qd, kd, vd, mode)

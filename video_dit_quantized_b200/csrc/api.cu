@@ -149,7 +149,32 @@ int launch_status(cudaError_t e) {
   return SAGE_ELAUNCH;
 }
 
+
 }  // namespace
+
+#ifdef SAGE_DEBUG
+std::mutex g_debug_mu;
+unsigned long long g_debug_first = 0;   // site << 48 | index of the last reported failure
+#endif
+
+// Debug build: waits for the call's work and turns any failed device-side
+// bounds check into SAGE_EBOUNDS.  Release build: returns rc unchanged.
+int debug_collect(cudaStream_t st, int rc) {
+#ifdef SAGE_DEBUG
+  if (rc != SAGE_OK) return rc;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE_ELAUNCH;
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  unsigned long long first = 0;
+  const unsigned w = debug_take_prepass(&first) | debug_take_attention(&first) | debug_take_ulysses(&first);
+  if (w) {
+    g_debug_first = first;
+    return SAGE_EBOUNDS;
+  }
+#else
+  (void)st;
+#endif
+  return rc;
+}
 
 bool encode_tmap_2d(void* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
@@ -216,8 +241,9 @@ int sage_quantize_qk_ex(const void* q, const void* k, const void* v, int B, int 
   if (scratch_bytes < prepass_scratch_bytes(B * H, N, d)) return SAGE_EWORKSPACE;
   if ((rc = check_device()) != SAGE_OK) return rc;
   const PrepassScratch s = prepass_scratch_carve(scratch, B * H, N, d);
-  return launch_status(launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale,
-                                      s, static_cast<cudaStream_t>(stream), q_granularity == 1));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return debug_collect(st, launch_status(launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+                                                        v_f8t, v_scale, s, st, q_granularity == 1)));
 }
 
 int sage_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
@@ -237,9 +263,10 @@ int sage_attn_quantized_ex(const int8_t* q_i8, const float* q_scale, const int8_
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAGE_EINVAL;
   if ((rc = check_device()) != SAGE_OK) return rc;
-  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d,
-                                        static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
-                                        static_cast<cudaStream_t>(stream), q_granularity == 1));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return debug_collect(st, launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N,
+                                                          d, static_cast<uint32_t*>(status), kDefaultTimeoutCycles, 0,
+                                                          st, q_granularity == 1)));
 }
 
 namespace sage {
@@ -261,8 +288,8 @@ int run_quantized(const void* q, const void* k, const void* v, void* o, int B, i
   cudaError_t e =
       launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s, st, qtok, in_map);
   if (e != cudaSuccess) return launch_status(e);
-  return launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N, d, status,
-                                        kDefaultTimeoutCycles, 0, st, qtok, o_map));
+  return debug_collect(st, launch_status(launch_attn_i8f8(q_i8, q_scale, k_i8, k_scale, v_f8t, v_scale, o, B * H, N,
+                                                          d, status, kDefaultTimeoutCycles, 0, st, qtok, o_map)));
 }
 }  // namespace
 }  // namespace sage
@@ -282,7 +309,8 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   if (mode == SAGE_MODE_BF16)
-    return launch_status(launch_attn_bf16(q, k, v, o, B * H, N, d, status, kDefaultTimeoutCycles, st));
+    return debug_collect(st, launch_status(launch_attn_bf16(q, k, v, o, B * H, N, d, status, kDefaultTimeoutCycles,
+                                                            st)));
   const RowMap plain{0, 0, 0, 0};
   return run_quantized(q, k, v, o, B, H, N, d, mode == SAGE_MODE_INT8_FP8_QTOKEN, ws, st, plain, plain);
 }
@@ -323,7 +351,8 @@ int sage_attn_fwd_seqpar(const void* q, const void* k, const void* v, void* o, i
     const cudaError_t e = launch_ulysses_permute(src[i], g[i], B, Nl, P * Hl, d, P, SAGE_ULYSSES_GATHER, 0, 0, st);
     if (e != cudaSuccess) return launch_status(e);
   }
-  return launch_status(launch_attn_bf16(g[0], g[1], g[2], o, B * Hl, N, d, status, kDefaultTimeoutCycles, st, chunks));
+  return debug_collect(st, launch_status(launch_attn_bf16(g[0], g[1], g[2], o, B * Hl, N, d, status,
+                                                          kDefaultTimeoutCycles, st, chunks)));
 }
 
 int sage_host_chunk_heads(int B, int H, int N, int d) {
@@ -573,8 +602,9 @@ int sage_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d
   if (rows * (d / 8) >= (1LL << 40)) return SAGE_EINVAL;
   const int rc = check_device();
   if (rc != SAGE_OK) return rc;
-  return launch_status(launch_ulysses_permute(src, dst, B, Nl, H, d, P, op, chunk_rows, base_rows,
-                                              static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return debug_collect(st, launch_status(launch_ulysses_permute(src, dst, B, Nl, H, d, P, op, chunk_rows, base_rows,
+                                                                st)));
 }
 
 int sage_dbg_mma_peak(int kind, int n, int iters, long long* cycles, int grid, void* status, void* stream) {
@@ -607,11 +637,46 @@ const char* sage_strerror(int code) {
     case SAGE_ELAUNCH: return "CUDA launch or runtime error";
     case SAGE_EWORKSPACE: return "workspace too small";
     case SAGE_ETIMEOUT: return "a bounded device-side wait ran out";
+    case SAGE_EBOUNDS: return "a device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
 
 int sage_device_check(void) { return check_device(); }
+
+int sage_debug_build(void) {
+#ifdef SAGE_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int sage_debug_last_failure(int* site, long long* index) {
+  if (!site || !index) return SAGE_EINVAL;
+#ifdef SAGE_DEBUG
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  *site = (int)(g_debug_first >> 48);
+  *index = (long long)(g_debug_first & 0xFFFFFFFFFFFFull);
+  return SAGE_OK;
+#else
+  *site = 0;
+  *index = 0;
+  return SAGE_EUNSUPPORTED;
+#endif
+}
+
+int sage_dbg_bounds_selftest(void* stream) {
+#ifdef SAGE_DEBUG
+  int rc = check_device();
+  if (rc != SAGE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return debug_collect(st, launch_status(launch_debug_selftest(st)));
+#else
+  (void)stream;
+  return SAGE_EUNSUPPORTED;
+#endif
+}
 
 int sage_dbg_qk_tiles(const int8_t* q_i8, const int8_t* k_i8, int B, int H, int N, int d, const int* tile_list, int n,
                       int32_t* out, void* stream) {

@@ -402,7 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qt < nT && gq < N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            if (SAGE_DCHECK((prm.o_map.row(bh, gq, N) * D + ch * 32) / 8 + v, (long long)gridDim.y * N * D / 8,
+                            kSiteAttnOut))
+              dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
     }
@@ -588,7 +591,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = softmax_c(D);
     float qs;
     if (qt < nT)
-      qs = prm.q_per_token ? prm.q_scale[(size_t)bh * prm.Npad + qt * 128 + row] : prm.q_scale[(size_t)bh * nT + qt];
+    {
+      const size_t qi = prm.q_per_token ? (size_t)bh * prm.Npad + qt * 128 + row : (size_t)bh * nT + qt;
+      const long long qe = (long long)gridDim.y * (prm.q_per_token ? prm.Npad : nT);
+      qs = SAGE_DCHECK(qi, qe, kSiteAttnQScale) ? prm.q_scale[qi] : 0.f;
+      (void)qe;
+    }
     else
       qs = 0.f;
     // p is produced already multiplied by the P scale 448 (2^(s - m + log2 448)),
@@ -597,13 +605,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // int32 S + 0x4B400000 read as a float is 12582912 + S exactly (|S| <= 127*127*128 < 2^22)
     constexpr uint32_t kMagicBits = 0x4B400000u;
     constexpr float kMagic = 12582912.0f;
-    float ks_next = prm.k_scale[(size_t)bh * nT];
+    const long long ks_ext = (long long)gridDim.y * nT;
+    (void)ks_ext;
+    float ks_next = SAGE_DCHECK((size_t)bh * nT, ks_ext, kSiteAttnKScale) ? prm.k_scale[(size_t)bh * nT] : 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t sr[128];
     for (int j = 0; j < nT && ok; ++j) {
       const float sc = __fmul_rn(__fmul_rn(qs, ks_next), c);
-      if (j + 1 < nT) ks_next = prm.k_scale[(size_t)bh * nT + j + 1];   // prefetch the next tile's scale
+      if (j + 1 < nT && SAGE_DCHECK((size_t)bh * nT + j + 1, ks_ext, kSiteAttnKScale))
+        ks_next = prm.k_scale[(size_t)bh * nT + j + 1];   // prefetch the next tile's scale
       if (!mbar_wait(&s_full[t], j & 1, abort_flag, limit)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
@@ -721,6 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int gq = qt * 128 + row;
       __nv_bfloat16* orow = prm.o + prm.o_map.row(bh, gq, N) * D;
       const float* vs = prm.v_scale + (size_t)bh * D;
+      const bool vs_ok = SAGE_DCHECK((size_t)bh * D + D - 1, (long long)gridDim.y * D, kSiteAttnVScale);
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t r[32];
@@ -729,14 +741,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t w[16];
 #pragma unroll
         for (int g = 0; g < 16; ++g) {
-          const float a0 = __fmul_rn(__uint_as_float(r[2 * g]), vs[ch * 32 + 2 * g]);
-          const float a1 = __fmul_rn(__uint_as_float(r[2 * g + 1]), vs[ch * 32 + 2 * g + 1]);
+          const float a0 = __fmul_rn(__uint_as_float(r[2 * g]), vs_ok ? vs[ch * 32 + 2 * g] : 0.f);
+          const float a1 = __fmul_rn(__uint_as_float(r[2 * g + 1]), vs_ok ? vs[ch * 32 + 2 * g + 1] : 0.f);
           w[g] = pack_bf16x2(__fdiv_rn(a0, l), __fdiv_rn(a1, l));   // l holds 448 * sum(p)
         }
         if (qt < nT && gq < N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            if (SAGE_DCHECK((prm.o_map.row(bh, gq, N) * D + ch * 32) / 8 + v, (long long)gridDim.y * N * D / 8,
+                            kSiteAttnOut))
+              dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
     }
@@ -975,6 +990,15 @@ cudaError_t launch_attn_bf16_d(const CUtensorMap& tq, const CUtensorMap& tk, con
 }
 
 }  // namespace
+
+unsigned debug_take_attention(unsigned long long* first) {
+#ifdef SAGE_DEBUG
+  return debug_take_tu(first);
+#else
+  (void)first;
+  return 0;
+#endif
+}
 
 cudaError_t launch_attn_i8f8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
                              const uint8_t* v_f8t, const float* v_scale, void* o, int BH, int N, int d,

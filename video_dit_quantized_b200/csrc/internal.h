@@ -13,6 +13,65 @@ constexpr int kTile = 128;
 // Bits OR-ed into the device status word.
 constexpr uint32_t kStatusTimeout = 1u;
 
+// ---- debug build (-DSAGE_DEBUG): device-side bounds checks ----------------
+// In a debug build every global access of the prepass, the attention
+// epilogue and scale loads, and the Ulysses permutations whose index is
+// computed checks the index against the extent of its buffer first.  A failed
+// check skips the access (nothing traps) and records itself in this
+// translation unit's debug word, with the site and index of the first
+// failure; the entry points of a debug build synchronise their stream and
+// return SAGE_EBOUNDS when any word is set.  A release build compiles every
+// check to `true`.  TMA loads need no check: the tensor maps bound them.
+#ifdef SAGE_DEBUG
+namespace dbg {
+static __device__ unsigned int g_word;            // one pair per translation unit
+static __device__ unsigned long long g_first;     // site << 48 | index of the first failure
+}  // namespace dbg
+__device__ __forceinline__ bool dcheck(long long idx, long long extent, unsigned site) {
+  if (idx >= 0 && idx < extent) return true;
+  atomicOr(&dbg::g_word, 1u);
+  atomicCAS(&dbg::g_first, 0ull, ((unsigned long long)site << 48) | ((unsigned long long)idx & 0xFFFFFFFFFFFFull));
+  return false;
+}
+#define SAGE_DCHECK(idx, extent, site) ::sage::dcheck((long long)(idx), (long long)(extent), (unsigned)(site))
+// Reads and clears this translation unit's words (host; after the work has
+// finished).  Returns the word; *first gets the first failure if it is 0.
+static inline unsigned debug_take_tu(unsigned long long* first) {
+  unsigned w = 0;
+  unsigned long long f = 0;
+  const unsigned zw = 0;
+  const unsigned long long zf = 0;
+  if (cudaMemcpyFromSymbol(&w, dbg::g_word, sizeof(w)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&f, dbg::g_first, sizeof(f)) != cudaSuccess)
+    return 1u;
+  cudaMemcpyToSymbol(dbg::g_word, &zw, sizeof(zw));
+  cudaMemcpyToSymbol(dbg::g_first, &zf, sizeof(zf));
+  if (w && first && *first == 0) *first = f;
+  return w;
+}
+#else
+#define SAGE_DCHECK(idx, extent, site) true
+#endif
+// Debug sites (the site field of a recorded failure).
+enum DebugSite : unsigned {
+  kSiteStatsIn = 1, kSiteStatsQ8, kSiteStatsQScale, kSiteStatsPartials,
+  kSiteFinIn, kSiteFinOut,
+  kSiteQuantIn, kSiteQuantPartials, kSiteQuantK8, kSiteQuantKScale, kSiteQuantV8,
+  kSiteAttnQScale = 20, kSiteAttnKScale, kSiteAttnVScale, kSiteAttnOut,
+  kSiteUlyssesSrc = 30, kSiteUlyssesDst,
+  kSiteSelftest = 99
+};
+// Per translation unit: reads and clears its debug words (0 in a release build).
+unsigned debug_take_prepass(unsigned long long* first);
+unsigned debug_take_attention(unsigned long long* first);
+unsigned debug_take_ulysses(unsigned long long* first);
+// A kernel that fails one check on purpose (the index equals the extent; no
+// memory is touched): the debug path's self-test.
+cudaError_t launch_debug_selftest(cudaStream_t stream);
+// Debug build: synchronises `st` and returns SAGE_EBOUNDS if a check failed
+// (rc when rc is already an error).  Release build: rc.
+int debug_collect(cudaStream_t st, int rc);
+
 inline int num_tiles(int N) { return (N + kTile - 1) / kTile; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -81,7 +81,8 @@ extern "C" int sage_quantize_qk_noalloc(const void* q, const void* k, const void
   // Every partial the kernels read is written earlier in the same call, so
   // nothing in the scratch has to start at zero.
   const PrepassScratch s = prepass_scratch_carve(base, B * H, N, d);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e = launch_prepass(q, k, v, B * H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, v_f8t, v_scale, s,
-                                       static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SAGE_OK : SAGE_ELAUNCH;
+                                       st);
+  return debug_collect(st, e == cudaSuccess ? SAGE_OK : SAGE_ELAUNCH);
 }

@@ -86,6 +86,10 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
   const int n0 = kb * kTile;
   const int nr = min(kTile, N - n0);
   const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
+  // buffer extents, for the checks of a debug build
+  const long long BHt = CHUNKED ? BHc : (int)gridDim.y;
+  const long long in_ext = BHt * N * V8, i8_ext = BHt * Npad * D / 8, part_ext = BHt * nK * D;
+  (void)in_ext; (void)i8_ext; (void)part_ext;
 
   if (threadIdx.x < D) vamax_s[threadIdx.x] = 0;
 
@@ -100,12 +104,14 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
     qv[i] = make_uint4(0, 0, 0, 0);
     if (row < nr) {
       const size_t at = CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e;
-      qv[i] = q[at];
-      ks[e] = k[at];
-      float y[8];
-      unpack8(v[at], y);
+      if (SAGE_DCHECK(at, in_ext, kSiteStatsIn)) {
+        qv[i] = q[at];
+        ks[e] = k[at];
+        float y[8];
+        unpack8(v[at], y);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) va[u] = fmaxf(va[u], fabsf(y[u]));
+        for (int u = 0; u < 8; ++u) va[u] = fmaxf(va[u], fabsf(y[u]));
+      }
     }
     float x[8];
     unpack8(qv[i], x);
@@ -122,7 +128,8 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
   uint2* qo = reinterpret_cast<uint2*>(q_i8 + ((size_t)bh * Npad + n0) * D);
   if constexpr (!TOKQ) {
     const float qinv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-    if (threadIdx.x == 0) q_scale[(size_t)bh * nK + kb] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
+    if (threadIdx.x == 0 && SAGE_DCHECK((size_t)bh * nK + kb, BHt * nK, kSiteStatsQScale))
+      q_scale[(size_t)bh * nK + kb] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.f;
 #pragma unroll
     for (int i = 0; i < PER_T; ++i) {
       const int e = threadIdx.x + i * kThreads;
@@ -131,7 +138,8 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
       int c[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) c[u] = qinv > 0.f ? quant_i8(x[u], qinv) : 0;
-      qo[e] = pack_i8x8(c);   // rows >= nr hold zeros (qv was zeroed)
+      if (SAGE_DCHECK(((size_t)bh * Npad + n0) * D / 8 + e, i8_ext, kSiteStatsQ8))
+        qo[e] = pack_i8x8(c);   // rows >= nr hold zeros (qv was zeroed)
     }
   } else {
     // the V8 consecutive lanes that hold one token reduce its absmax
@@ -146,11 +154,13 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
 #pragma unroll
       for (int o = V8 / 2; o > 0; o >>= 1) ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, o));
       const float rinv = ra > 0.f ? __fdiv_rn(127.0f, ra) : 0.f;
-      if (e % V8 == 0) q_scale[(size_t)bh * Npad + n0 + e / V8] = ra > 0.f ? __fdiv_rn(ra, 127.0f) : 0.f;
+      if (e % V8 == 0 && SAGE_DCHECK((size_t)bh * Npad + n0 + e / V8, BHt * Npad, kSiteStatsQScale))
+        q_scale[(size_t)bh * Npad + n0 + e / V8] = ra > 0.f ? __fdiv_rn(ra, 127.0f) : 0.f;
       int c[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) c[u] = rinv > 0.f ? quant_i8(x[u], rinv) : 0;
-      qo[e] = pack_i8x8(c);   // rows >= nr: zero codes and scale 0
+      if (SAGE_DCHECK(((size_t)bh * Npad + n0) * D / 8 + e, i8_ext, kSiteStatsQ8))
+        qo[e] = pack_i8x8(c);   // rows >= nr: zero codes and scale 0
     }
   }
   __syncthreads();
@@ -168,10 +178,12 @@ __global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __
       mn = fminf(mn, x);
       mx = fmaxf(mx, x);
     }
-    scr.k_psum[pidx + c] = s;
-    scr.k_pmin[pidx + c] = mn;
-    scr.k_pmax[pidx + c] = mx;
-    scr.v_pamax[pidx + c] = __int_as_float(vamax_s[c]);
+    if (SAGE_DCHECK(pidx + c, part_ext, kSiteStatsPartials)) {
+      scr.k_psum[pidx + c] = s;
+      scr.k_pmin[pidx + c] = mn;
+      scr.k_pmax[pidx + c] = mx;
+      scr.v_pamax[pidx + c] = __int_as_float(vamax_s[c]);
+    }
   }
 }
 
@@ -190,13 +202,17 @@ __global__ void __launch_bounds__(64) prepass_finalize_kernel(int N, int nK, Pre
   const int bh = blockIdx.x;
   const int c = blockIdx.y * 32 + (threadIdx.x & 31);
   const size_t col = (size_t)bh * nK * D + c;       // partial (bh, block 0, c); block t is t * D further
+  const long long part_ext = (long long)gridDim.x * nK * D, out_ext = (long long)gridDim.x * D;
+  (void)part_ext; (void)out_ext;
   if (threadIdx.x < 32) {
     const double* gs = scr.k_psum + col;
     double total = 0.0;
     double A[kFinBatch], B[kFinBatch];
     auto load = [&](double(&r)[kFinBatch], int t0) {
 #pragma unroll
-      for (int i = 0; i < kFinBatch; ++i) r[i] = t0 + i < nK ? gs[(size_t)(t0 + i) * D] : 0.0;
+      for (int i = 0; i < kFinBatch; ++i)
+        r[i] = t0 + i < nK && SAGE_DCHECK(col + (size_t)(t0 + i) * D, part_ext, kSiteFinIn) ? gs[(size_t)(t0 + i) * D]
+                                                                                           : 0.0;
     };
     auto add = [&](const double(&r)[kFinBatch], int t0) {
 #pragma unroll
@@ -210,14 +226,17 @@ __global__ void __launch_bounds__(64) prepass_finalize_kernel(int N, int nK, Pre
       load(A, t0 + 2 * kFinBatch);
       add(B, t0 + kFinBatch);
     }
-    k_mean[(size_t)bh * D + c] = __double2float_rn(__ddiv_rn(total, (double)N));
+    if (SAGE_DCHECK((size_t)bh * D + c, out_ext, kSiteFinOut))
+      k_mean[(size_t)bh * D + c] = __double2float_rn(__ddiv_rn(total, (double)N));
   } else {
     const float* ga = scr.v_pamax + col;
     float a = 0.f;
     float A[kFinBatch], B[kFinBatch];
     auto load = [&](float(&r)[kFinBatch], int t0) {
 #pragma unroll
-      for (int i = 0; i < kFinBatch; ++i) r[i] = t0 + i < nK ? ga[(size_t)(t0 + i) * D] : 0.f;
+      for (int i = 0; i < kFinBatch; ++i)
+        r[i] = t0 + i < nK && SAGE_DCHECK(col + (size_t)(t0 + i) * D, part_ext, kSiteFinIn) ? ga[(size_t)(t0 + i) * D]
+                                                                                           : 0.f;
     };
     auto take = [&](const float(&r)[kFinBatch]) {
 #pragma unroll
@@ -230,8 +249,10 @@ __global__ void __launch_bounds__(64) prepass_finalize_kernel(int N, int nK, Pre
       load(A, t0 + 2 * kFinBatch);
       take(B);
     }
-    v_scale[(size_t)bh * D + c] = a > 0.f ? __fdiv_rn(a, 448.0f) : 0.f;
-    scr.v_amax[(size_t)bh * D + c] = a;
+    if (SAGE_DCHECK((size_t)bh * D + c, out_ext, kSiteFinOut)) {
+      v_scale[(size_t)bh * D + c] = a > 0.f ? __fdiv_rn(a, 448.0f) : 0.f;
+      scr.v_amax[(size_t)bh * D + c] = a;
+    }
   }
 }
 
@@ -261,21 +282,30 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   const int nr = min(kTile, N - n0);
   const size_t in_base = ((size_t)bh * N + n0) * V8;  // plain layout, in uint4
   const size_t pidx = ((size_t)bh * nK + kb) * D;
+  // buffer extents, for the checks of a debug build
+  const long long BHt = CHUNKED ? BHc : (int)gridDim.y;
+  const long long in_ext = BHt * N * V8, i8_ext = BHt * Npad * D / 8, part_ext = BHt * nK * D, ch_ext = BHt * D;
+  (void)in_ext; (void)i8_ext; (void)part_ext; (void)ch_ext;
 
   // k_scale of this block from the partial min / max: fp32 subtraction is
   // monotone, so max|fl(x - m)| over the block is attained at its min or max.
   float kam = 0.f;
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
-    const float m = k_mean[(size_t)bh * D + c];
+    float m = 0.f, a = 0.f;
+    if (SAGE_DCHECK((size_t)bh * D + c, ch_ext, kSiteQuantPartials)) {
+      m = k_mean[(size_t)bh * D + c];
+      a = scr.v_amax[(size_t)bh * D + c];
+    }
     mean_s[c] = m;
-    kam = fmaxf(fabsf(__fsub_rn(scr.k_pmax[pidx + c], m)), fabsf(__fsub_rn(scr.k_pmin[pidx + c], m)));
-    const float a = scr.v_amax[(size_t)bh * D + c];
+    if (SAGE_DCHECK(pidx + c, part_ext, kSiteQuantPartials))
+      kam = fmaxf(fabsf(__fsub_rn(scr.k_pmax[pidx + c], m)), fabsf(__fsub_rn(scr.k_pmin[pidx + c], m)));
     vinv_s[c] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
   }
   kam = block_max(kam, red);   // contains __syncthreads
   const float kinv = kam > 0.f ? __fdiv_rn(127.0f, kam) : 0.f;
-  if (threadIdx.x == 0) k_scale[(size_t)bh * nK + kb] = kam > 0.f ? __fdiv_rn(kam, 127.0f) : 0.f;
+  if (threadIdx.x == 0 && SAGE_DCHECK((size_t)bh * nK + kb, BHt * nK, kSiteQuantKScale))
+    k_scale[(size_t)bh * nK + kb] = kam > 0.f ? __fdiv_rn(kam, 127.0f) : 0.f;
 
   // ---- K: smoothed INT8 codes ----
   uint2* ko = reinterpret_cast<uint2*>(k_i8 + ((size_t)bh * Npad + n0) * D);
@@ -285,12 +315,15 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
     const int row = e / V8, c0 = (e % V8) * 8;
     int c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (row < nr && kinv > 0.f) {
-      float x[8];
-      unpack8(k[CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e], x);
+      const size_t at = CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e;
+      if (SAGE_DCHECK(at, in_ext, kSiteQuantIn)) {
+        float x[8];
+        unpack8(k[at], x);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
+        for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
+      }
     }
-    ko[e] = pack_i8x8(c);
+    if (SAGE_DCHECK(((size_t)bh * Npad + n0) * D / 8 + e, i8_ext, kSiteQuantK8)) ko[e] = pack_i8x8(c);
   }
 
   // ---- V: stage the block, then e4m3 codes written channel-major ----
@@ -298,8 +331,8 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   for (int i = 0; i < PER_T; ++i) {
     const int e = threadIdx.x + i * kThreads;
     const int row = e / V8;
-    vs[e] = row < nr ? v[CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e]
-                     : make_uint4(0, 0, 0, 0);
+    const size_t at = row < nr ? (CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e) : 0;
+    vs[e] = row < nr && SAGE_DCHECK(at, in_ext, kSiteQuantIn) ? v[at] : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(vs);
@@ -321,8 +354,9 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
       w[g] = inv > 0.f ? pack_e4m3x4(x[0], x[1], x[2], x[3]) : 0u;
     }
     // padding tokens (n >= nr) were staged as +0 and encode to 0x00
-    uint4* dst = reinterpret_cast<uint4*>(v_f8t + ((size_t)bh * D + c) * Npad + (size_t)n0 + chunk * 16);
-    *dst = make_uint4(w[0], w[1], w[2], w[3]);
+    const size_t off = ((size_t)bh * D + c) * Npad + (size_t)n0 + chunk * 16;   // bytes, a multiple of 16
+    if (SAGE_DCHECK(off / 16, BHt * D * Npad / 16, kSiteQuantV8))
+      *reinterpret_cast<uint4*>(v_f8t + off) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -356,7 +390,26 @@ cudaError_t launch_prepass_d(const void* q, const void* k, const void* v, int BH
   return cudaGetLastError();
 }
 
+__global__ void debug_selftest_kernel() {
+  // one check that fails (index == extent); nothing is read or written
+  (void)SAGE_DCHECK(1, 1, kSiteSelftest);
+}
+
 }  // namespace
+
+unsigned debug_take_prepass(unsigned long long* first) {
+#ifdef SAGE_DEBUG
+  return debug_take_tu(first);
+#else
+  (void)first;
+  return 0;
+#endif
+}
+
+cudaError_t launch_debug_selftest(cudaStream_t stream) {
+  debug_selftest_kernel<<<1, 1, 0, stream>>>();
+  return cudaGetLastError();
+}
 
 size_t prepass_scratch_bytes(int BH, int N, int d) {
   const size_t n = (size_t)BH * num_tiles(N) * d;

@@ -32,6 +32,7 @@ namespace {
 struct UlyGeom {
   long long B, Nl, H, Hl, P, N;
   long long chunk_rows, base_rows;  // of the [P] side
+  long long src_rows, dst_rows;     // extents of the two buffers, in rows (checks of a debug build)
 };
 
 // Row of the [P] side holding (chunk r, b, token n of the chunk, head hl).
@@ -77,10 +78,21 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
   const long long i = t / VPR;
   if (i >= rows) return;
   const int v = (int)(t % VPR);
-  dst[dst_row(i, op, g) * VPR + v] = src[src_row(i, op, g) * VPR + v];
+  const long long si = src_row(i, op, g) * VPR + v, di = dst_row(i, op, g) * VPR + v;
+  if (SAGE_DCHECK(si, g.src_rows * VPR, kSiteUlyssesSrc) && SAGE_DCHECK(di, g.dst_rows * VPR, kSiteUlyssesDst))
+    dst[di] = src[si];
 }
 
 }  // namespace
+
+unsigned debug_take_ulysses(unsigned long long* first) {
+#ifdef SAGE_DEBUG
+  return debug_take_tu(first);
+#else
+  (void)first;
+  return 0;
+#endif
+}
 
 cudaError_t launch_ulysses_permute(const void* src, void* dst, int B, int Nl, int H, int d, int P, int op,
                                    long long chunk_rows, long long base_rows, cudaStream_t stream) {
@@ -94,6 +106,11 @@ cudaError_t launch_ulysses_permute(const void* src, void* dst, int B, int Nl, in
   g.chunk_rows = chunk_rows > 0 ? chunk_rows : (long long)B * g.Hl * Nl;
   g.base_rows = base_rows;
   const long long rows = (long long)B * Nl * H;
+  // the [P] side spans base_rows + (P - 1) * chunk_rows + one chunk; the other side is dense
+  const long long p_rows = g.base_rows + (g.P - 1) * g.chunk_rows + (long long)B * g.Hl * Nl;
+  const bool p_is_dst = op == 0 || op == 3;
+  g.src_rows = p_is_dst ? rows : p_rows;
+  g.dst_rows = p_is_dst ? p_rows : rows;
   const int vpr = d * 2 / 16;
   const long long threads = rows * vpr;
   const unsigned grid = (unsigned)((threads + 255) / 256);

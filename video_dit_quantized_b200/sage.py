@@ -21,7 +21,7 @@ DTYPE_F32 = 1
 BLK = 128
 P_SCALE = 448.0
 
-OK, EINVAL, EUNSUPPORTED, ELAUNCH, EWORKSPACE, ETIMEOUT = 0, -1, -2, -3, -4, -5
+OK, EINVAL, EUNSUPPORTED, ELAUNCH, EWORKSPACE, ETIMEOUT, EBOUNDS = 0, -1, -2, -3, -4, -5, -6
 SELECT_EVERY_ITERATION, SELECT_MEAN = 0, 1
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sage.h")
@@ -33,10 +33,10 @@ class SageError(RuntimeError):
         super().__init__(f"{what}: {strerror(code)} ({code})")
 
 
-def _load() -> ctypes.CDLL:
-    path = _build.LIB_PATH
+def load_library(path: str) -> ctypes.CDLL:
+    """Loads a build of the library (libsage.so, or libsage_debug.so) with the C prototypes set."""
     if not os.path.exists(path):
-        raise ImportError(f"libsage.so is not built ({path}); run video_dit_quantized_b200.build.build()")
+        raise ImportError(f"{os.path.basename(path)} is not built ({path}); run video_dit_quantized_b200.build.build()")
     lib = ctypes.CDLL(path)
     vp, i32, sz, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
     sig = {
@@ -73,6 +73,9 @@ def _load() -> ctypes.CDLL:
         "sage_attn_fwd_seqpar": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]),
         "sage_host_chunk_heads": (i32, [i32, i32, i32, i32]),
         "sage_host_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+        "sage_debug_build": (i32, []),
+        "sage_debug_last_failure": (i32, [vp, vp]),
+        "sage_dbg_bounds_selftest": (i32, [vp]),
         "sage_dbg_mma_peak": (i32, [i32, i32, i32, vp, i32, vp, vp]),
         "sage_dbg_linear_bf16_forced_timeout": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, vp, ll, vp]),
     }
@@ -83,7 +86,17 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-LIB = _load()
+LIB = load_library(_build.LIB_PATH)
+_DEBUG_LIB = None
+
+
+def debug_library() -> ctypes.CDLL:
+    """libsage_debug.so (the same sources built with SAGE_DEBUG: device-side bounds checks, entry points
+    that synchronise and return EBOUNDS), loaded once; raises ImportError if it is not built."""
+    global _DEBUG_LIB
+    if _DEBUG_LIB is None:
+        _DEBUG_LIB = load_library(_build.DEBUG_LIB_PATH)
+    return _DEBUG_LIB
 
 
 def header_functions() -> list[str]:
