@@ -67,7 +67,7 @@ DEFAULT_WORKLOAD = "wan14b_720p"
 # of the same shape, scaled by heads (each head's operands are read from DRAM
 # once).  Keyed by (workload, H, mode); absent keys report null.
 NCU_TRAFFIC_BYTES = {
-    ("wan14b_720p", 40, "int8_fp8"): 1.651e9,
+    ("wan14b_720p", 40, "int8_fp8"): 1.650e9,
     ("wan14b_720p", 40, "bf16"): 3.006e9,
 }
 # Linear GEMM DRAM bytes per launch (ncu captures of the same kernels at the
