@@ -184,6 +184,18 @@ def test_host_chunk_rule():
     assert sage.host_chunk_heads(1, 2, 1024, 96) == 0             # bad shape
 
 
+def test_host_workspace_is_two_chunk_workspaces():
+    """sage_attn_fwd_host keeps two chunks in flight, each with its own workspace half."""
+    def one(B, H, N, d, mode, chunk):
+        return (sage.workspace_bytes(1, chunk, N, d, mode) + 255) // 256 * 256
+    for mode in (sage.MODE_INT8_FP8, sage.MODE_INT8_FP8_QTOKEN, sage.MODE_BF16):
+        assert sage.host_workspace_bytes(1, 40, 75600, 128, mode, 0) == 2 * one(1, 40, 75600, 128, mode, 2)
+        assert sage.host_workspace_bytes(2, 5, 1500, 64, mode, 3) == 2 * one(2, 5, 1500, 64, mode, 3)
+        assert sage.host_workspace_bytes(1, 1, 1000, 128, mode, 0) == one(1, 1, 1000, 128, mode, 1)   # one chunk
+    assert sage.host_workspace_bytes(1, 2, 1024, 96, sage.MODE_BF16, 0) == 0          # bad shape
+    assert sage.host_workspace_bytes(1, 2, 1024, 128, 7, 0) == 0                      # bad mode
+
+
 def test_binding_checks_what_the_c_abi_cannot_see():
     """dtype, contiguity and shape of tensor arguments are checked before any device call (CPU tensors)."""
     import torch
