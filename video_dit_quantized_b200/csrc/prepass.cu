@@ -287,6 +287,23 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
   const long long in_ext = BHt * N * V8, i8_ext = BHt * Npad * D / 8, part_ext = BHt * nK * D, ch_ext = BHt * D;
   (void)in_ext; (void)i8_ext; (void)part_ext; (void)ch_ext;
 
+  // the block's K and V rows go in flight first; the scales below only need
+  // the per-head and per-block statistics
+  uint4 kr[PER_T], vr[PER_T];
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int e = threadIdx.x + i * kThreads;
+    const int row = e / V8;
+    kr[i] = vr[i] = make_uint4(0, 0, 0, 0);
+    if (row < nr) {
+      const size_t at = CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e;
+      if (SAGE_DCHECK(at, in_ext, kSiteQuantIn)) {
+        kr[i] = k[at];
+        vr[i] = v[at];
+      }
+    }
+  }
+
   // k_scale of this block from the partial min / max: fp32 subtraction is
   // monotone, so max|fl(x - m)| over the block is attained at its min or max.
   float kam = 0.f;
@@ -315,25 +332,17 @@ __global__ void __launch_bounds__(kThreads) prepass_quant_kv_kernel(const uint4*
     const int row = e / V8, c0 = (e % V8) * 8;
     int c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (row < nr && kinv > 0.f) {
-      const size_t at = CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e;
-      if (SAGE_DCHECK(at, in_ext, kSiteQuantIn)) {
-        float x[8];
-        unpack8(k[at], x);
+      float x[8];
+      unpack8(kr[i], x);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
-      }
+      for (int u = 0; u < 8; ++u) c[u] = quant_i8(__fsub_rn(x[u], mean_s[c0 + u]), kinv);
     }
     if (SAGE_DCHECK(((size_t)bh * Npad + n0) * D / 8 + e, i8_ext, kSiteQuantK8)) ko[e] = pack_i8x8(c);
   }
 
-  // ---- V: stage the block, then e4m3 codes written channel-major ----
+  // ---- V: stage the block (padding rows +0), then e4m3 codes written channel-major ----
 #pragma unroll
-  for (int i = 0; i < PER_T; ++i) {
-    const int e = threadIdx.x + i * kThreads;
-    const int row = e / V8;
-    const size_t at = row < nr ? (CHUNKED ? (size_t)in_map.row(bh, n0 + row, N) * V8 + (e % V8) : in_base + e) : 0;
-    vs[e] = row < nr && SAGE_DCHECK(at, in_ext, kSiteQuantIn) ? v[at] : make_uint4(0, 0, 0, 0);
-  }
+  for (int i = 0; i < PER_T; ++i) vs[threadIdx.x + i * kThreads] = vr[i];
   __syncthreads();
   const __nv_bfloat16* vh = reinterpret_cast<const __nv_bfloat16*>(vs);
   constexpr int PAIRS = D * (kTile / 16);   // (channel, 16-token chunk)
