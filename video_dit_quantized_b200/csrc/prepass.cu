@@ -64,7 +64,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // grid (nK, BH), or (nK * BH) with the head fastest when CHUNKED.  TOKQ: Q gets one scale per token (q_scale [BH, Npad]) instead
 // of one per 128-token block (q_scale [BH, nK]).
 template <int D, bool TOKQ, bool CHUNKED>
-__global__ void __launch_bounds__(kThreads) prepass_stats_kernel(const uint4* __restrict__ q,
+__global__ void __launch_bounds__(kThreads, 3) prepass_stats_kernel(const uint4* __restrict__ q,
                                                                  const uint4* __restrict__ k,
                                                                  const uint4* __restrict__ v, int N, int Npad,
                                                                  int8_t* __restrict__ q_i8,
