@@ -171,10 +171,10 @@ def test_quantized_per_token_q_small_all_rows(w, cuda_dev):
     assert torch.equal(o_b.view(torch.int16), o.view(torch.int16))
 
 
-def test_quantized_per_token_q_full_size_sampled(cuda_dev, big_inputs):
+@pytest.mark.parametrize("name", ["cogvideox2b", "wan1.3b_480p", "wan14b_720p"])
+def test_quantized_per_token_q_full_size_sampled(name, cuda_dev, big_inputs):
     import torch
     from video_dit_quantized_b200 import sage
-    name = "wan1.3b_480p"
     w = synth.WORKLOADS[name]
     q, k, v, qd, kd, vd = big_inputs(name)
     hs = [0, w.H - 1]

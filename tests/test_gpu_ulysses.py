@@ -60,16 +60,19 @@ def test_permutes_match_reference(B, Nl, H, d, P, cuda_dev):
     assert torch.equal(back.view(torch.int16), x.view(torch.int16))       # RECV_O inverts SEND
 
 
-@pytest.mark.parametrize("mode_name,P,Nl,Hl,d", [("int8_fp8", 8, 1181, 2, 128), ("int8_fp8", 3, 333, 3, 64),
-                                                 ("int8_fp8_qtoken", 4, 257, 2, 128), ("bf16", 8, 1181, 2, 128),
-                                                 ("bf16", 1, 640, 4, 64), ("int8_fp8", 1, 1000, 3, 128)])
-def test_seqpar_equals_plain_attention(mode_name, P, Nl, Hl, d, cuda_dev):
-    """The fused chunk-layout call gives bitwise the plain call's output on the gathered heads."""
+@pytest.mark.parametrize("mode_name,P,Nl,Hl,d,B", [("int8_fp8", 8, 1181, 2, 128, 1), ("int8_fp8", 3, 333, 3, 64, 1),
+                                                   ("int8_fp8_qtoken", 4, 257, 2, 128, 1),
+                                                   ("bf16", 8, 1181, 2, 128, 1), ("bf16", 1, 640, 4, 64, 1),
+                                                   ("int8_fp8", 1, 1000, 3, 128, 1), ("int8_fp8", 2, 300, 3, 64, 2),
+                                                   ("int8_fp8_qtoken", 3, 129, 1, 128, 3), ("bf16", 2, 200, 2, 128, 2)])
+def test_seqpar_equals_plain_attention(mode_name, P, Nl, Hl, d, B, cuda_dev):
+    """The fused chunk-layout call gives bitwise the plain call's output on the gathered heads
+    (several batch elements too: the chunk rows interleave b and the local heads)."""
     import torch
     from video_dit_quantized_b200 import sage
     mode = {"int8_fp8": sage.MODE_INT8_FP8, "int8_fp8_qtoken": sage.MODE_INT8_FP8_QTOKEN,
             "bf16": sage.MODE_BF16}[mode_name]
-    B, N, H = 1, P * Nl, P * Hl
+    N, H = P * Nl, P * Hl
     w = synth.Workload("sp", B, Hl, N, d, seed=P * 10 + Hl, outlier_frac=0.01)
     q, k, v = (_bf16(a, cuda_dev) for a in synth.qkv_numpy(w))             # plain [B, Hl, N, d]
     scat = lambda t: ulysses_ref_permute(t, torch.empty((P, B, Nl, Hl, d), dtype=t.dtype, device=cuda_dev),
