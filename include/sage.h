@@ -187,7 +187,7 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
  *   memory is needed for the copies to overlap.
  * q_dev, k_dev, v_dev, o_dev: device staging buffers bf16 [B,H,N,d] (caller-owned).
  * workspace: at least sage_host_workspace_bytes(B, H, N, d, mode, chunk_heads)
- *   bytes, zero-filled before the first call: its two halves (each rounded
+ *   bytes, 256-byte aligned, zero-filled before the first call: its two halves (each rounded
  *   down to 256 bytes; one when B*H == 1) are the workspaces of alternate
  *   chunks, each with its status word first, at the same offsets whatever the
  *   mode, so one buffer serves calls of every mode.

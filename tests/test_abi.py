@@ -276,3 +276,15 @@ def test_binding_signatures_match_the_header():
         assert f.argtypes is not None, name
         assert [a for a in f.argtypes] == [_ctype(p) for p in params], name
         assert f.restype == _ctype(ret), name
+
+
+def test_host_entry_rejects_a_workspace_off_256_bytes():
+    """The host pipeline hands each half of its workspace to sage_attn_fwd (256-byte aligned); a buffer
+    aligned to 16 bytes only is refused before any copy or launch (the addresses are never touched)."""
+    B, H, N, d = 1, 2, 1000, 128
+    p16 = ctypes.c_void_p(0x10000010)          # 16-byte aligned, not 256
+    p256 = ctypes.c_void_p(0x10000100)
+    n = sage.host_workspace_bytes(B, H, N, d, sage.MODE_INT8_FP8, 0)
+    rc = sage.LIB.sage_attn_fwd_host(p256, p256, p256, p256, B, H, N, d, sage.MODE_INT8_FP8, p256, p256, p256, p256,
+                                     p16, n, 0, None)
+    assert rc == sage.EINVAL

@@ -391,6 +391,8 @@ int sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_hos
   const void* ptrs[] = {q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return SAGE_EINVAL;
+  // each chunk workspace is handed to sage_attn_fwd, which wants 256-byte alignment
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_EINVAL;
   const int BH = B * H;
   if (chunk_heads <= 0) chunk_heads = sage_host_chunk_heads(B, H, N, d);
   if (chunk_heads > BH) chunk_heads = BH;
