@@ -220,6 +220,24 @@ def cpu_baseline(w, n_rows: int, impl_line: bool = False):
             "seconds": dt}
 
 
+def attention_config(w, args, world: int) -> dict:
+    """The config of an attention line; the reference arm prints the same one."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
+            "global_batch": world * w.B, "parallelism": f"independent calls x{world}",
+            "l2": "inputs (2.3 GB) larger than L2; no flush"}
+
+
+def linear_config(w, world: int) -> dict:
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "global_batch": world,
+            "parallelism": f"independent calls x{world}", "l2": "X (774 MB bf16) larger than L2; no flush"}
+
+
+def stack_config(base, world: int) -> dict:
+    return {"workload": "layer_stack", "layers": synth.LAYER_STACK_LAYERS, "B": base.B, "H": base.H, "N": base.N,
+            "d": base.d, "full_precision_layers": list(synth.LAYER_STACK_FULL_PRECISION), "seeds": "layer index",
+            "parallelism": f"independent stacks x{world}", "l2": "every layer's inputs (1.0 GB) larger than L2; no flush"}
+
+
 def run_reference_linear(args, rank, world):
     """Reference arm of --op linear: the CPU oracle on a bounded sample per step."""
     w = synth.LINEAR_WORKLOADS[args.linear_workload]
@@ -237,7 +255,7 @@ def run_reference_linear(args, rank, world):
         "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int64 block sums, f32 (CPU oracle)", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "sample": "256 sampled rows per step"},
+        "config": linear_config(w, world),
         "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": r["cores"], "kind": "oracle", "sample": r["sample"]},
         "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -261,13 +279,13 @@ def run_reference(args, rank, world):
         vals.append(r["value"])
         secs.append(r["seconds"])
     tflops = statistics.median(vals)
+    metric = "attention TFLOPS per call (4*B*H*N^2*d)" + (", 40-layer selective stack" if args.op == "stack" else "")
     line = {
-        "impl": "reference", "metric": "attention TFLOPS per call (4*B*H*N^2*d)", "value": tflops,
+        "impl": "reference", "metric": metric, "value": tflops,
         "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
-                   "sample": f"1 head, {rows} sampled query rows per step"},
+        "config": stack_config(w, world) if args.op == "stack" else attention_config(w, args, world),
         "cpu_baseline": {"value": tflops, "unit": "TFLOPS", "cores": r["cores"], "kind": "oracle",
                          "sample": r["sample"]},
         "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -424,9 +442,7 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/fp8e4m3 (fp32 accumulate)" if quant else "bf16 (fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mode": args.mode,
-                   "global_batch": world * w.B, "parallelism": f"independent calls x{world}",
-                   "l2": "inputs (2.3 GB) larger than L2; no flush"},
+        "config": attention_config(w, args, world),
         "kernels_ms": {"prepass_median": statistics.median(prep_ms), "attention_median": statistics.median(attn_ms),
                        "attention_p10": float(np.percentile(attn_ms, 10)),
                        "attention_p90": float(np.percentile(attn_ms, 90)),
@@ -602,9 +618,7 @@ def run_linear(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "int8 (int32 block sums, fp32 accumulate)" if lmode == "w8a8" else "bf16 (fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "global_batch": world,
-                   "parallelism": f"independent calls x{world}",
-                   "l2": "X (774 MB bf16) larger than L2; no flush"},
+        "config": linear_config(w, world),
         "kernels_ms": {("quantize_median" if lmode == "w8a8" else "dequantize_median"): statistics.median(quant_ms),
                        "gemm_median": statistics.median(gemm_ms),
                        "gemm_min": min(gemm_ms), "gemm_max": max(gemm_ms)},
@@ -788,10 +802,7 @@ def run_stack(args, rank, world, local_rank):
         "value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/fp8e4m3 + bf16 layers (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": "layer_stack", "layers": L, "B": base.B, "H": base.H, "N": base.N, "d": base.d,
-                   "full_precision_layers": list(synth.LAYER_STACK_FULL_PRECISION), "seeds": "layer index",
-                   "parallelism": f"independent stacks x{world}",
-                   "l2": "every layer's inputs (1.0 GB) larger than L2; no flush"},
+        "config": stack_config(base, world),
         "by_mode": by_mode,
         "all_bf16_stack": {"ms_per_step": ms_bf16, "tflops": flops / (ms_bf16 * 1e-3) / 1e12,
                            "speedup_of_selective": ms_bf16 / ms, "clocks": clocks_bf16},
